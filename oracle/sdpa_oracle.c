@@ -1,0 +1,299 @@
+/*
+ * CPU oracle for multi-head scaled-dot-product attention — TEST INFRASTRUCTURE ONLY.
+ *
+ * Only the test suite, the smoke check and the CPU-baseline leg of the benchmark may load
+ * this file's library. The CUDA library never includes, links or calls it, and it shares
+ * no code, header, table or constant with the CUDA library.
+ *
+ * What it computes is the plain definition from the Flux.jl page "Neural Network
+ * primitives from NNlib.jl", entry NNlib.scaled_dot_product_attention:
+ *
+ *   out = softmax(scale * query' * key + bias, masked) * value        (first paragraph)
+ *
+ * in float64, one output row at a time, with a two-pass softmax and no tiling. Each
+ * step below names the argument of that entry which defines it.
+ *
+ * Layout. The page's arrays are column-major (head_dim, nheads, seq_len, batch), which is
+ * the same memory as row-major [batch][seq][head][dim]; this file indexes row-major:
+ *   q[b][i][h][c]   (batch, q_len, nheads, qk_head_dim)
+ *   k[b][j][g][c]   (batch, kv_len, nkvheads, qk_head_dim)
+ *   v[b][j][g][e]   (batch, kv_len, nkvheads, v_head_dim)
+ *   out[b][i][h][e] (batch, q_len, nheads, v_head_dim)
+ * The bias and the mask are broadcastable to the page's (kv_len, q_len, nheads, batch);
+ * they are addressed through four element strides in that order (key j, query i, head h,
+ * batch b), a stride of 0 meaning the array is broadcast along that axis.
+ *
+ * Readings where the page leaves a step open (each also listed in the design notes):
+ *  - GQA head sharing: query head h uses key/value head h / (nheads/nkvheads) (contiguous
+ *    groups). The other grouping, h % nkvheads, is selectable for tests.
+ *  - A masked logit is -infinity, so its weight is exactly zero; the bias is added first.
+ *  - The bias is not multiplied by the scale.
+ *  - A query row that attends to no key is NaN; a query row at or past q_lengths[b] is 0,
+ *    and the zero wins when both hold.
+ *  - :bottom_right takes q_offset[b] = kv_len[b] - q_len[b], with the array sizes where the
+ *    lengths are not given; a negative offset is allowed.
+ *
+ * Parity pins: every function here is pinned by the CPU tests (closed forms, the stated
+ * equivalences of the entry, PyTorch's float64 CPU routine on the special cases it can
+ * express, brute force on tiny inputs).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_RANGE 2
+#define ORACLE_ERR_NOMEM 3
+
+typedef struct {
+  int64_t batch, q_len, kv_len, nheads, nkvheads, dqk, dv;
+  double scale;               /* NaN: 1/sqrt(dqk) (argument `scale`) */
+  int32_t causal;             /* 0 false, 1 true (top-left), 2 :bottom_right */
+  int32_t kv_head_rule;       /* 0: h / (nheads/nkvheads); 1: h % nkvheads */
+  int64_t q_offset_scalar;    /* used when q_offset == NULL */
+  const int64_t* q_offset;    /* [batch] or NULL */
+  const int64_t* q_lengths;   /* [batch] or NULL (= q_len for every batch element) */
+  const int64_t* kv_lengths;  /* [batch] or NULL (= kv_len for every batch element) */
+  const double* bias;         /* NULL or broadcast array */
+  int64_t bias_stride[4];     /* (j, i, h, b) element strides */
+  const uint8_t* mask;        /* NULL or broadcast boolean array (0 = not attended) */
+  int64_t mask_stride[4];     /* (j, i, h, b) element strides */
+} oracle_sdpa_problem;
+
+/* Checks the shape rules the entry states: nheads divisible by nkvheads (GQA paragraph). */
+static int check_problem(const oracle_sdpa_problem* p) {
+  if (!p) return ORACLE_ERR_ARG;
+  if (p->batch < 0 || p->q_len < 0 || p->kv_len < 0) return ORACLE_ERR_ARG;
+  if (p->nheads <= 0 || p->nkvheads <= 0 || p->dqk <= 0 || p->dv <= 0) return ORACLE_ERR_ARG;
+  if (p->nheads % p->nkvheads != 0) return ORACLE_ERR_ARG;
+  if (p->causal < 0 || p->causal > 2) return ORACLE_ERR_ARG;
+  if (p->kv_head_rule < 0 || p->kv_head_rule > 1) return ORACLE_ERR_ARG;
+  return ORACLE_OK;
+}
+
+/* One output row: batch b, query head h, query position i. `s` is scratch of kv_len doubles. */
+static void sdpa_row(const oracle_sdpa_problem* p, const double* q, const double* k,
+                     const double* v, double* out, int64_t b, int64_t h, int64_t i,
+                     double* s, unsigned char* allowed) {
+  const int64_t Lq = p->q_len, Lk = p->kv_len, H = p->nheads, Hkv = p->nkvheads;
+  const int64_t D = p->dqk, Dv = p->dv;
+  double* o = out + ((b * Lq + i) * H + h) * Dv;
+
+  /* Argument `q_lengths`: the output is zero at the queries past q_lengths[b]. */
+  const int64_t qlen_b = p->q_lengths ? p->q_lengths[b] : Lq;
+  if (i >= qlen_b) {
+    for (int64_t e = 0; e < Dv; ++e) o[e] = 0.0;
+    return;
+  }
+  /* Argument `kv_lengths`: the keys past kv_lengths[b] are not attended to. */
+  const int64_t kvlen_b = p->kv_lengths ? p->kv_lengths[b] : Lk;
+
+  /* GQA paragraph: key/value heads are shared across query heads. */
+  const int64_t group = H / Hkv;
+  const int64_t g = (p->kv_head_rule == 0) ? (h / group) : (h % Hkv);
+
+  /* Argument `is_causal` / `q_offset`: query i attends keys j <= q_offset + i. */
+  int64_t off = 0;
+  if (p->causal == 1) off = p->q_offset ? p->q_offset[b] : p->q_offset_scalar;
+  if (p->causal == 2) off = kvlen_b - qlen_b;
+
+  /* Argument `scale`: default 1/sqrt(qk_head_dim). */
+  const double scale = isnan(p->scale) ? 1.0 / sqrt((double)D) : p->scale;
+
+  const double* qi = q + ((b * Lq + i) * H + h) * D;
+  int64_t n_allowed = 0;
+  double m = -INFINITY;
+  for (int64_t j = 0; j < Lk; ++j) {
+    /* `mask`, `is_causal` and `kv_lengths` combine: attended only where all allow it. */
+    int ok = (j < kvlen_b);
+    if (p->causal != 0 && !(j <= off + i)) ok = 0;
+    if (p->mask) {
+      const uint8_t mv = p->mask[j * p->mask_stride[0] + i * p->mask_stride[1] +
+                                 h * p->mask_stride[2] + b * p->mask_stride[3]];
+      if (!mv) ok = 0;
+    }
+    allowed[j] = (unsigned char)ok;
+    if (!ok) continue;
+    const double* kj = k + ((b * Lk + j) * Hkv + g) * D;
+    double dot = 0.0;
+    for (int64_t c = 0; c < D; ++c) dot += qi[c] * kj[c];
+    double x = scale * dot;
+    /* Argument `bias`: added to the logits before the softmax (not scaled). */
+    if (p->bias)
+      x += p->bias[j * p->bias_stride[0] + i * p->bias_stride[1] + h * p->bias_stride[2] +
+                   b * p->bias_stride[3]];
+    s[j] = x;
+    if (x > m) m = x;
+    ++n_allowed;
+  }
+
+  /* A query attending to no key has a NaN output (fused-implementation paragraph). */
+  if (n_allowed == 0) {
+    for (int64_t e = 0; e < Dv; ++e) o[e] = NAN;
+    return;
+  }
+
+  /* Softmax over the attended keys, then the weighted sum of the values. */
+  double denom = 0.0;
+  for (int64_t j = 0; j < Lk; ++j) {
+    if (!allowed[j]) continue;
+    s[j] = exp(s[j] - m);
+    denom += s[j];
+  }
+  for (int64_t e = 0; e < Dv; ++e) o[e] = 0.0;
+  for (int64_t j = 0; j < Lk; ++j) {
+    if (!allowed[j]) continue;
+    const double w = s[j] / denom;
+    const double* vj = v + ((b * Lk + j) * Hkv + g) * Dv;
+    for (int64_t e = 0; e < Dv; ++e) o[e] += w * vj[e];
+  }
+}
+
+/* scaled_dot_product_attention(query, key, value, [bias]; mask, scale, is_causal, q_offset,
+ * q_lengths, kv_lengths): every (b, h, i) row of the output. */
+int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const double* k,
+                        const double* v, double* out) {
+  int rc = check_problem(p);
+  if (rc) return rc;
+  if (p->batch == 0 || p->q_len == 0) return ORACLE_OK;
+  const int64_t rows = p->batch * p->nheads * p->q_len;
+  int failed = 0;
+#pragma omp parallel
+  {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(p->kv_len > 0 ? p->kv_len : 1));
+    unsigned char* allowed = (unsigned char*)malloc((size_t)(p->kv_len > 0 ? p->kv_len : 1));
+    if (!s || !allowed) {
+#pragma omp atomic write
+      failed = 1;
+    } else {
+#pragma omp for schedule(dynamic, 16)
+      for (int64_t r = 0; r < rows; ++r) {
+        const int64_t b = r / (p->nheads * p->q_len);
+        const int64_t h = (r / p->q_len) % p->nheads;
+        const int64_t i = r % p->q_len;
+        sdpa_row(p, q, k, v, out, b, h, i, s, allowed);
+      }
+    }
+    free(s);
+    free(allowed);
+  }
+  return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* Writing new keys/values into a KV cache at a per-sequence position (the Keras issue
+ * "MultiHeadAttention is missing a position_bias call argument": `cache_update_index`; the
+ * Flax discussion's cached_key/cached_value, shaped (batch, len, heads, head_dim)):
+ *   cache[b][index[b] + t][g][c] = new[b][t][g][c]   for t < n_new.
+ * An index outside [0, capacity - n_new] is an error and nothing is written. */
+int oracle_cache_update_at_index(double* cache, const double* new_rows, int64_t batch,
+                                 int64_t capacity, int64_t n_new, int64_t nkvheads, int64_t d,
+                                 const int64_t* index) {
+  if (batch < 0 || capacity < 0 || n_new < 0 || nkvheads <= 0 || d <= 0 || !index)
+    return ORACLE_ERR_ARG;
+  for (int64_t b = 0; b < batch; ++b)
+    if (index[b] < 0 || index[b] + n_new > capacity) return ORACLE_ERR_RANGE;
+  const int64_t row = nkvheads * d;
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t t = 0; t < n_new; ++t)
+      memcpy(cache + (b * capacity + index[b] + t) * row, new_rows + (b * n_new + t) * row,
+             sizeof(double) * (size_t)row);
+  return ORACLE_OK;
+}
+
+/* Decoding with a KV cache (the entry's example "decoding with a KV cache"): write the new
+ * keys/values at index[b], then attend with is_causal=:bottom_right and
+ * kv_lengths[b] = index[b] + n_new, the n_new queries being the last positions. */
+int oracle_sdpa_decode_with_cache(const oracle_sdpa_problem* p_in, const double* q,
+                                  const double* k_new, const double* v_new, double* k_cache,
+                                  double* v_cache, const int64_t* index, double* out) {
+  if (!p_in || !index) return ORACLE_ERR_ARG;
+  oracle_sdpa_problem p = *p_in; /* q_len = n_new, kv_len = capacity */
+  int rc = oracle_cache_update_at_index(k_cache, k_new, p.batch, p.kv_len, p.q_len, p.nkvheads,
+                                        p.dqk, index);
+  if (rc) return rc;
+  rc = oracle_cache_update_at_index(v_cache, v_new, p.batch, p.kv_len, p.q_len, p.nkvheads, p.dv,
+                                    index);
+  if (rc) return rc;
+  int64_t* kvl = (int64_t*)malloc(sizeof(int64_t) * (size_t)(p.batch > 0 ? p.batch : 1));
+  if (!kvl) return ORACLE_ERR_NOMEM;
+  for (int64_t b = 0; b < p.batch; ++b) kvl[b] = index[b] + p.q_len;
+  p.kv_lengths = kvl;
+  p.q_lengths = NULL;
+  p.causal = 2;
+  rc = oracle_sdpa_forward(&p, q, k_cache, v_cache, out);
+  free(kvl);
+  return rc;
+}
+
+/* Block classification of a boolean mask, after the splash-attention mask info of the JAX
+ * pull request "Support dynamic masks in splash attention": the mask is cut into blocks of
+ * bq queries x bk keys, and each block is empty (no key attended), full (every key
+ * attended) or partial. A block at the ragged edge counts only its in-range cells.
+ *
+ * Outputs, for mask heads h < nheads (the mask's own head extent) and block rows qb:
+ *  - cls[h][qb][kb]: 0 empty, 1 partial, 2 full (this library's own encoding);
+ *  - count[h][qb]: the number of non-empty blocks of the row;
+ *  - list[h][qb][n] for n < count: the non-empty kb in increasing order, with the class in
+ *    the top two bits: kb | (cls << 30);
+ *  - bits: for each partial block, at block slot (h*nqb + qb)*nkb + kb, bq rows of
+ *    ceil(bk/32) 32-bit words, bit c of word w of row r = mask(h, qb*bq + r, kb*bk + 32w + c);
+ *    out-of-range cells are 0. Slots of non-partial blocks are left untouched.
+ * The mask is read as mask[j*ms[0] + i*ms[1] + h*ms[2]] (key j, query i, head h). */
+int oracle_block_mask_info(const uint8_t* mask, const int64_t ms[3], int64_t nheads,
+                           int64_t q_len, int64_t kv_len, int64_t bq, int64_t bk, uint8_t* cls,
+                           int32_t* count, uint32_t* list, uint32_t* bits) {
+  if (!mask || !ms || nheads <= 0 || q_len <= 0 || kv_len <= 0 || bq <= 0 || bk <= 0)
+    return ORACLE_ERR_ARG;
+  const int64_t nqb = (q_len + bq - 1) / bq, nkb = (kv_len + bk - 1) / bk;
+  const int64_t words = (bk + 31) / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t hq = 0; hq < nheads * nqb; ++hq) {
+    const int64_t h = hq / nqb, qb = hq % nqb;
+    int32_t n = 0;
+    for (int64_t kb = 0; kb < nkb; ++kb) {
+      int64_t cells = 0, set = 0;
+      for (int64_t r = 0; r < bq; ++r) {
+        const int64_t i = qb * bq + r;
+        if (i >= q_len) break;
+        for (int64_t c = 0; c < bk; ++c) {
+          const int64_t j = kb * bk + c;
+          if (j >= kv_len) break;
+          ++cells;
+          if (mask[j * ms[0] + i * ms[1] + h * ms[2]]) ++set;
+        }
+      }
+      const uint8_t cl = (set == 0) ? 0 : (set == cells ? 2 : 1);
+      cls[(h * nqb + qb) * nkb + kb] = cl;
+      if (cl != 0) list[(h * nqb + qb) * nkb + (n++)] = (uint32_t)kb | ((uint32_t)cl << 30);
+      if (cl == 1) {
+        uint32_t* blk = bits + ((h * nqb + qb) * nkb + kb) * bq * words;
+        for (int64_t r = 0; r < bq; ++r)
+          for (int64_t w = 0; w < words; ++w) {
+            uint32_t word = 0;
+            for (int64_t c = 0; c < 32; ++c) {
+              const int64_t i = qb * bq + r, jc = w * 32 + c, j = kb * bk + jc;
+              if (i < q_len && jc < bk && j < kv_len && mask[j * ms[0] + i * ms[1] + h * ms[2]])
+                word |= (1u << c);
+            }
+            blk[r * words + w] = word;
+          }
+      }
+    }
+    count[h * nqb + qb] = n;
+  }
+  return ORACLE_OK;
+}
+
+/* Number of host threads the OpenMP loops above use (reported beside timings). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

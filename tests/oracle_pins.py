@@ -1,0 +1,501 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Every pin checks the oracle against something the page or mathematics fixes: a closed form,
+an equivalence the entry states, PyTorch's float64 CPU routine on the special cases it can
+express, or brute-force counting. Each takes the oracle library handle, so that the mutant
+tests can run the same pins against deliberately broken builds of the oracle.
+
+Passages cited are from the Flux.jl page "Neural Network primitives from NNlib.jl", entry
+NNlib.scaled_dot_product_attention, unless stated otherwise.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+PINS = []
+
+
+def pin(fn):
+    PINS.append(fn)
+    return fn
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _qkv(rng, B, Lq, Lk, H, Hkv, D, Dv=None):
+    Dv = Dv or D
+    q = rng.standard_normal((B, Lq, H, D))
+    k = rng.standard_normal((B, Lk, Hkv, D))
+    v = rng.standard_normal((B, Lk, Hkv, Dv))
+    return q, k, v
+
+
+def _torch_sdpa(q, k, v, **kw):
+    """PyTorch's float64 CPU scaled_dot_product_attention in our layout. PyTorch's layout is
+    (batch, nheads, seq, dim), so the seq and head axes are swapped on the way in and out
+    (the entry's layout paragraph warns of exactly this permutation)."""
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).permute(0, 2, 1, 3)
+    am = kw.pop("attn_mask", None)
+    if am is not None:
+        am = torch.from_numpy(np.ascontiguousarray(am))
+    out = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=am, **kw)
+    return out.permute(0, 2, 1, 3).numpy()
+
+
+def _close(a, b, tol=1e-12):
+    np.testing.assert_allclose(a, b, rtol=0, atol=tol)
+
+
+# ---- library routine on the special cases it expresses ------------------------------------
+
+@pin
+def torch_plain_unequal_lengths_dv(lib):
+    """First paragraph: softmax(scale·qᵀk)·v with the default scale 1/√qk_head_dim, and a
+    value head size different from the query's (Returns: (v_head_dim, nheads, q_len, ...))."""
+    q, k, v = _qkv(_rng(11), 2, 5, 7, 3, 3, 8, 6)
+    _close(oracle.sdpa_forward(q, k, v, lib=lib), _torch_sdpa(q, k, v))
+
+
+@pin
+def torch_causal_top_left(lib):
+    """Argument is_causal=true: query i attends keys j ≤ i (q_offset 0), for equal and for
+    unequal lengths; PyTorch's is_causal is the same top-left alignment."""
+    for (Lq, Lk) in ((6, 6), (4, 9), (9, 4)):
+        q, k, v = _qkv(_rng(12 + Lq), 2, Lq, Lk, 2, 2, 8)
+        _close(oracle.sdpa_forward(q, k, v, is_causal=True, lib=lib),
+               _torch_sdpa(q, k, v, is_causal=True))
+
+
+@pin
+def torch_gqa(lib):
+    """GQA paragraph: fewer key/value heads shared across query heads; PyTorch's enable_gqa
+    repeats each key/value head over a contiguous group of query heads."""
+    q, k, v = _qkv(_rng(13), 2, 5, 6, 8, 2, 8)
+    _close(oracle.sdpa_forward(q, k, v, lib=lib), _torch_sdpa(q, k, v, enable_gqa=True))
+
+
+@pin
+def torch_bool_mask_broadcast(lib):
+    """Argument mask: a boolean array broadcastable to (kv_len, q_len, nheads, batch), i.e.
+    row-major (batch, nheads, q_len, kv_len); false entries are not attended."""
+    rng = _rng(14)
+    q, k, v = _qkv(rng, 2, 5, 7, 3, 3, 8)
+    mask = rng.random((1, 3, 5, 7)) < 0.6  # broadcast over batch
+    mask[..., 0] = True  # keep one key per row
+    _close(oracle.sdpa_forward(q, k, v, mask=mask, lib=lib),
+           _torch_sdpa(q, k, v, attn_mask=np.broadcast_to(mask, (2, 3, 5, 7)).copy()))
+
+
+@pin
+def torch_float_bias_and_scale(lib):
+    """Arguments bias and scale: the bias is added to the scaled logits before the softmax."""
+    rng = _rng(15)
+    q, k, v = _qkv(rng, 2, 4, 6, 2, 2, 8)
+    bias = rng.standard_normal((2, 1, 4, 6))  # broadcast over heads
+    _close(oracle.sdpa_forward(q, k, v, bias=bias, scale=0.37, lib=lib),
+           _torch_sdpa(q, k, v, attn_mask=bias, scale=0.37))
+
+
+# ---- closed forms -------------------------------------------------------------------------
+
+@pin
+def closed_form_two_keys(lib):
+    """With two keys the softmax is a logistic function: w0 = 1/(1+exp(x1-x0)), where
+    x = scale·qᵀk + bias (arguments scale and bias)."""
+    rng = _rng(21)
+    q, k, v = _qkv(rng, 1, 1, 2, 1, 1, 4, 3)
+    bias = np.array([[[[0.8, -1.3]]]])
+    s = 0.5
+    x0 = s * float(q[0, 0, 0] @ k[0, 0, 0]) + 0.8
+    x1 = s * float(q[0, 0, 0] @ k[0, 1, 0]) - 1.3
+    w0 = 1.0 / (1.0 + math.exp(x1 - x0))
+    expect = w0 * v[0, 0, 0] + (1.0 - w0) * v[0, 1, 0]
+    _close(oracle.sdpa_forward(q, k, v, bias=bias, scale=s, lib=lib)[0, 0, 0], expect)
+
+
+@pin
+def default_scale_uses_qk_dim(lib):
+    """Argument scale: nothing means 1/√(qk_head_dim), even when v_head_dim differs."""
+    q, k, v = _qkv(_rng(22), 1, 3, 4, 1, 1, 9, 4)
+    _close(oracle.sdpa_forward(q, k, v, lib=lib), oracle.sdpa_forward(q, k, v, scale=1 / 3.0, lib=lib))
+
+
+@pin
+def rows_sum_to_one(lib):
+    """The softmax weights of a row sum to one: with every value equal to 1 the output is 1,
+    whatever the bias, mask, causal alignment and lengths."""
+    rng = _rng(23)
+    q, k, _ = _qkv(rng, 3, 5, 9, 4, 2, 8)
+    v = np.ones((3, 9, 2, 5))
+    mask = rng.random((3, 4, 5, 9)) < 0.7
+    mask[..., 0] = True
+    bias = 3.0 * rng.standard_normal((1, 4, 5, 9))
+    out = oracle.sdpa_forward(q, k, v, bias=bias, mask=mask, is_causal=True, q_offset=[0, 2, 4],
+                              kv_lengths=[9, 5, 7], lib=lib)
+    _close(out, np.ones_like(out))
+
+
+@pin
+def weights_readout_is_a_distribution(lib):
+    """With kv_len ≤ v_head_dim and value[j] = e_j, the output row is the weight row: it is
+    non-negative, sums to one and is exactly zero on the keys that are not attended."""
+    rng = _rng(24)
+    Lk = 6
+    q, k, _ = _qkv(rng, 1, 4, Lk, 1, 1, 8)
+    v = np.eye(Lk)[None, :, None, :]
+    mask = rng.random((1, 1, 4, Lk)) < 0.6
+    mask[..., 1] = True
+    w = oracle.sdpa_forward(q, k, v, mask=mask, lib=lib)[0, :, 0, :]
+    assert (w >= 0).all()
+    _close(w.sum(axis=-1), np.ones(4))
+    assert (w[~mask[0, 0]] == 0).all()
+
+
+@pin
+def single_key_returns_its_value(lib):
+    """With one attended key the weight is 1 and the output is that key's value: kv_lengths=1,
+    and row 0 of is_causal=true (q_offset 0) sees only key 0."""
+    q, k, v = _qkv(_rng(25), 2, 3, 5, 2, 1, 4, 6)
+    out = oracle.sdpa_forward(q, k, v, kv_lengths=[1, 1], lib=lib)
+    for b in range(2):
+        for h in range(2):
+            _close(out[b, :, h], np.broadcast_to(v[b, 0, 0], (3, 6)), 1e-15)
+    out = oracle.sdpa_forward(q, k, v, is_causal=True, lib=lib)
+    _close(out[:, 0, :, :], np.broadcast_to(v[:, 0:1, 0, :], (2, 2, 6)), 1e-15)
+
+
+@pin
+def identical_keys_average_values(lib):
+    """All keys equal: every weight is 1/n over the n attended keys, so the output is the
+    mean of their values (kv_lengths decides n)."""
+    rng = _rng(26)
+    q = rng.standard_normal((2, 3, 2, 4))
+    k = np.broadcast_to(rng.standard_normal((1, 1, 1, 4)), (2, 6, 1, 4)).copy()
+    v = rng.standard_normal((2, 6, 1, 5))
+    out = oracle.sdpa_forward(q, k, v, kv_lengths=[4, 6], lib=lib)
+    _close(out[0], np.broadcast_to(v[0, :4, 0].mean(0), (3, 2, 5)))
+    _close(out[1], np.broadcast_to(v[1, :6, 0].mean(0), (3, 2, 5)))
+
+
+# ---- equivalences the entry states ---------------------------------------------------------
+
+@pin
+def causal_equals_make_causal_mask(lib):
+    """is_causal=true equals mask = make_causal_mask(query; dims=3) for equal lengths: the
+    mask is true where key j ≤ query i."""
+    q, k, v = _qkv(_rng(31), 2, 7, 7, 2, 2, 8)
+    i = np.arange(7)[:, None]
+    j = np.arange(7)[None, :]
+    causal_mask = (j <= i)[None, None]
+    _close(oracle.sdpa_forward(q, k, v, is_causal=True, lib=lib),
+           oracle.sdpa_forward(q, k, v, mask=causal_mask, lib=lib))
+
+
+@pin
+def bottom_right_printed_example(lib):
+    """Examples, KV-cache decoding: :bottom_right with kv_lengths [13,23,33,43] and 3 queries
+    equals is_causal=true with q_offset [10,20,30,40] (sizes from the printed example)."""
+    ex = json.load(open(os.path.join(GOLDEN, "printed_examples.json")))["examples"][3]
+    D, H, Lq, B = ex["query"]
+    _, Hk, Lk, _ = ex["key"]
+    rng = _rng(32)
+    q = rng.random((B, Lq, H, D))  # rand(Float32, ...) in the example: uniform [0, 1)
+    k = rng.random((B, Lk, Hk, D))
+    v = k  # k = v = rand(...) in the example
+    a = oracle.sdpa_forward(q, k, v, is_causal="bottom_right", kv_lengths=ex["kv_lengths"], lib=lib)
+    b = oracle.sdpa_forward(q, k, v, is_causal=True, q_offset=ex["equivalent_q_offset"],
+                            kv_lengths=ex["kv_lengths"], lib=lib)
+    _close(a, b, 0.0)
+    assert a.shape == tuple(reversed(ex["output"]))
+    # and the first new query attends exactly the keys 0 .. q_offset[b]
+    c = oracle.sdpa_forward(q[:, :1], k, v, kv_lengths=np.array(ex["equivalent_q_offset"]) + 1, lib=lib)
+    _close(a[:, :1], c)
+
+
+@pin
+def bottom_right_defaults_to_array_sizes(lib):
+    """:bottom_right with no lengths: q_offset = kv_len - q_len of the arrays; with equal
+    lengths it is the top-left mask."""
+    q, k, v = _qkv(_rng(33), 2, 3, 8, 2, 2, 4)
+    _close(oracle.sdpa_forward(q, k, v, is_causal="bottom_right", lib=lib),
+           oracle.sdpa_forward(q, k, v, is_causal=True, q_offset=5, lib=lib), 0.0)
+    q, k, v = _qkv(_rng(34), 2, 6, 6, 2, 2, 4)
+    _close(oracle.sdpa_forward(q, k, v, is_causal="bottom_right", lib=lib),
+           oracle.sdpa_forward(q, k, v, is_causal=True, lib=lib), 0.0)
+
+
+@pin
+def bottom_right_with_q_lengths(lib):
+    """:bottom_right takes q_offset = kv_lengths - q_lengths per batch element when both are
+    given; the last valid query then attends all kv_lengths keys."""
+    q, k, v = _qkv(_rng(35), 2, 5, 9, 2, 2, 4)
+    out = oracle.sdpa_forward(q, k, v, is_causal="bottom_right", q_lengths=[3, 5],
+                              kv_lengths=[7, 9], lib=lib)
+    ref = oracle.sdpa_forward(q, k, v, is_causal=True, q_offset=[4, 4], q_lengths=[3, 5],
+                              kv_lengths=[7, 9], lib=lib)
+    _close(out, ref, 0.0)
+    full = oracle.sdpa_forward(q, k, v, kv_lengths=[7, 9], lib=lib)
+    _close(out[0, 2], full[0, 2])
+    _close(out[1, 4], full[1, 4])
+
+
+@pin
+def gqa_equals_repeated_heads(lib):
+    """GQA paragraph: sharing key/value heads across query heads equals repeating each of them
+    over its group of nheads/nkvheads consecutive query heads."""
+    q, k, v = _qkv(_rng(36), 2, 4, 5, 6, 2, 4)
+    _close(oracle.sdpa_forward(q, k, v, lib=lib),
+           oracle.sdpa_forward(q, np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2), lib=lib))
+    _close(oracle.sdpa_forward(q, k, v, kv_head_rule="interleaved", lib=lib),
+           oracle.sdpa_forward(q, np.tile(k, (1, 1, 3, 1)), np.tile(v, (1, 1, 3, 1)), lib=lib))
+
+
+@pin
+def kv_lengths_equal_truncation(lib):
+    """Argument kv_lengths: keys past kv_lengths[b] are not attended, which equals the call on
+    arrays cut to that length (the padded-batch example)."""
+    q, k, v = _qkv(_rng(37), 3, 4, 9, 2, 2, 4)
+    lens = [3, 9, 6]
+    out = oracle.sdpa_forward(q, k, v, kv_lengths=lens, lib=lib)
+    for b, n in enumerate(lens):
+        _close(out[b:b + 1], oracle.sdpa_forward(q[b:b + 1], k[b:b + 1, :n], v[b:b + 1, :n], lib=lib))
+    # an integer applies to every batch element
+    _close(oracle.sdpa_forward(q, k, v, kv_lengths=5, lib=lib),
+           oracle.sdpa_forward(q, k[:, :5], v[:, :5], lib=lib))
+
+
+@pin
+def q_lengths_zero_rows(lib):
+    """Argument q_lengths: the output is zero at the queries past q_lengths[b]; earlier rows
+    are unchanged."""
+    q, k, v = _qkv(_rng(38), 2, 6, 5, 2, 2, 4)
+    out = oracle.sdpa_forward(q, k, v, q_lengths=[2, 6], lib=lib)
+    full = oracle.sdpa_forward(q, k, v, lib=lib)
+    assert (out[0, 2:] == 0).all()
+    _close(out[0, :2], full[0, :2], 0.0)
+    _close(out[1], full[1], 0.0)
+
+
+@pin
+def mask_causal_lengths_combine_by_and(lib):
+    """mask, is_causal and kv_lengths combine: a key is attended only where all allow it, which
+    equals one explicit mask that is their conjunction."""
+    rng = _rng(39)
+    q, k, v = _qkv(rng, 2, 6, 8, 2, 2, 4)
+    mask = rng.random((2, 2, 6, 8)) < 0.7
+    mask[..., 0] = True
+    off = [1, 2]
+    lens = [5, 8]
+    i = np.arange(6)[:, None]
+    j = np.arange(8)[None, :]
+    combined = np.stack([mask[b] & (j <= off[b] + i)[None] & (j < lens[b])[None] for b in range(2)])
+    _close(oracle.sdpa_forward(q, k, v, mask=mask, is_causal=True, q_offset=off, kv_lengths=lens, lib=lib),
+           oracle.sdpa_forward(q, k, v, mask=combined, lib=lib))
+
+
+@pin
+def mask_equals_minus_infinity_bias(lib):
+    """A false mask entry removes the key exactly as a bias of -infinity does; an all-true mask
+    changes nothing."""
+    rng = _rng(40)
+    q, k, v = _qkv(rng, 2, 4, 7, 2, 2, 4)
+    mask = rng.random((2, 2, 4, 7)) < 0.5
+    mask[..., 3] = True
+    bias = np.where(mask, 0.0, -np.inf)
+    _close(oracle.sdpa_forward(q, k, v, mask=mask, lib=lib), oracle.sdpa_forward(q, k, v, bias=bias, lib=lib))
+    _close(oracle.sdpa_forward(q, k, v, mask=np.ones((1, 1, 1, 1), bool), lib=lib),
+           oracle.sdpa_forward(q, k, v, lib=lib), 0.0)
+
+
+@pin
+def bias_row_shift_invariance(lib):
+    """Adding a constant per query row to the bias leaves the softmax unchanged."""
+    rng = _rng(41)
+    q, k, v = _qkv(rng, 2, 4, 6, 2, 2, 4)
+    bias = rng.standard_normal((2, 2, 4, 6))
+    shift = rng.standard_normal((2, 2, 4, 1)) * 5
+    _close(oracle.sdpa_forward(q, k, v, bias=bias, lib=lib),
+           oracle.sdpa_forward(q, k, v, bias=bias + shift, lib=lib), 1e-11)
+
+
+@pin
+def bias_is_per_head_and_batch(lib):
+    """The bias is indexed by head and batch: a bias that differs only in head 1 / batch 1
+    changes only those output rows, and a bias of a single key row equals a large logit."""
+    rng = _rng(42)
+    q, k, v = _qkv(rng, 2, 3, 5, 2, 2, 4)
+    bias = np.zeros((2, 2, 3, 5))
+    bias[1, 1, :, 2] = 80.0  # weight of key 2 becomes ~1 for batch 1, head 1
+    out = oracle.sdpa_forward(q, k, v, bias=bias, lib=lib)
+    ref = oracle.sdpa_forward(q, k, v, lib=lib)
+    _close(out[0], ref[0], 0.0)
+    _close(out[1, :, 0], ref[1, :, 0], 0.0)
+    _close(out[1, :, 1], np.broadcast_to(v[1, 2, 1], (3, 4)), 1e-9)
+
+
+@pin
+def scale_equivalence(lib):
+    """Argument scale multiplies qᵀk: scaling the query by a equals scaling `scale` by a."""
+    q, k, v = _qkv(_rng(43), 2, 4, 6, 2, 2, 4)
+    _close(oracle.sdpa_forward(2.5 * q, k, v, scale=0.3, lib=lib),
+           oracle.sdpa_forward(q, k, v, scale=0.75, lib=lib))
+
+
+@pin
+def empty_row_is_nan_and_padding_wins(lib):
+    """A query that attends to no key has a NaN output (fused-implementation paragraph); a
+    query past q_lengths is zero even then."""
+    q, k, v = _qkv(_rng(44), 1, 3, 4, 1, 1, 4)
+    mask = np.ones((1, 1, 3, 4), bool)
+    mask[0, 0, 1, :] = False
+    mask[0, 0, 2, :] = False
+    out = oracle.sdpa_forward(q, k, v, mask=mask, q_lengths=[2], lib=lib)
+    assert np.isfinite(out[0, 0]).all()
+    assert np.isnan(out[0, 1]).all()
+    assert (out[0, 2] == 0).all()
+    # a negative causal offset leaves the first rows without keys
+    out = oracle.sdpa_forward(q, k, v, is_causal=True, q_offset=-2, lib=lib)
+    assert np.isnan(out[0, :2]).all() and np.isfinite(out[0, 2]).all()
+
+
+@pin
+def printed_example_shapes(lib):
+    """Examples: the output has size (v_head_dim, nheads, q_len, batch) for the plain, GQA
+    and padded calls."""
+    ex = json.load(open(os.path.join(GOLDEN, "printed_examples.json")))["examples"]
+    rng = _rng(45)
+    for e in ex[:3]:
+        qs, ks, vs = (tuple(reversed(e[n])) for n in ("query", "key", "value"))
+        out = oracle.sdpa_forward(rng.random(qs), rng.random(ks), rng.random(vs),
+                                  kv_lengths=e.get("kv_lengths"), lib=lib)
+        assert out.shape == tuple(reversed(e["output"]))
+        assert np.isfinite(out).all()
+
+
+# ---- cache update and decode ----------------------------------------------------------------
+
+@pin
+def cache_update_writes_only_the_new_rows(lib):
+    """Keras issue on MultiHeadAttention, cache_update_index: the new keys/values are written
+    at the given position of each sequence; every other cache entry is unchanged."""
+    rng = _rng(51)
+    cache = rng.standard_normal((3, 10, 2, 4))
+    new = rng.standard_normal((3, 2, 2, 4))
+    idx = [0, 5, 8]
+    out = oracle.cache_update_at_index(cache, new, idx, lib=lib)
+    expect = cache.copy()
+    for b, i in enumerate(idx):
+        expect[b, i:i + 2] = new[b]
+    _close(out, expect, 0.0)
+    try:
+        oracle.cache_update_at_index(cache, new, [0, 5, 9], lib=lib)
+    except oracle.OracleError:
+        pass
+    else:
+        raise AssertionError("an index past capacity - n_new must be rejected")
+
+
+@pin
+def decode_equals_attention_over_the_grown_cache(lib):
+    """Decoding example: after writing the new key/value at index[b], :bottom_right attention
+    of one new query equals plain attention over the index[b] + 1 keys of the cache."""
+    rng = _rng(52)
+    B, cap, H, Hkv, D = 3, 12, 4, 2, 8
+    q = rng.standard_normal((B, 1, H, D))
+    kn, vn = rng.standard_normal((B, 1, Hkv, D)), rng.standard_normal((B, 1, Hkv, D))
+    kc, vc = rng.standard_normal((B, cap, Hkv, D)), rng.standard_normal((B, cap, Hkv, D))
+    idx = np.array([0, 6, 11])
+    out, kc2, vc2 = oracle.sdpa_decode_with_cache(q, kn, vn, kc, vc, idx, lib=lib)
+    for b in range(B):
+        n = idx[b] + 1
+        kk = np.concatenate([kc[b:b + 1, :idx[b]], kn[b:b + 1]], axis=1)
+        vv = np.concatenate([vc[b:b + 1, :idx[b]], vn[b:b + 1]], axis=1)
+        _close(out[b:b + 1], oracle.sdpa_forward(q[b:b + 1], kk, vv, lib=lib))
+        _close(kc2[b, :n], kk[0], 0.0)
+    # several new queries: the t-th attends the keys up to index[b] + t
+    q3 = rng.standard_normal((B, 3, H, D))
+    kn3, vn3 = rng.standard_normal((B, 3, Hkv, D)), rng.standard_normal((B, 3, Hkv, D))
+    idx3 = np.array([0, 4, 9])
+    out3, kc3, vc3 = oracle.sdpa_decode_with_cache(q3, kn3, vn3, kc, vc, idx3, lib=lib)
+    for b in range(B):
+        for t in range(3):
+            n = idx3[b] + t + 1
+            _close(out3[b:b + 1, t:t + 1],
+                   oracle.sdpa_forward(q3[b:b + 1, t:t + 1], kc3[b:b + 1, :n], vc3[b:b + 1, :n], lib=lib))
+
+
+# ---- block classification --------------------------------------------------------------------
+
+def _decode_info(info, H, Lq, Lk, bq, bk):
+    """Rebuild the dense mask from the classes and the packed partial bits."""
+    m = np.zeros((H, Lq, Lk), dtype=np.uint8)
+    nqb, nkb = info["cls"].shape[1:]
+    for h in range(H):
+        for qb in range(nqb):
+            for kb in range(nkb):
+                c = info["cls"][h, qb, kb]
+                r0, c0 = qb * bq, kb * bk
+                r1, c1 = min(Lq, r0 + bq), min(Lk, c0 + bk)
+                if c == 2:
+                    m[h, r0:r1, c0:c1] = 1
+                elif c == 1:
+                    words = info["bits"][h, qb, kb]
+                    for r in range(r1 - r0):
+                        for cc in range(c1 - c0):
+                            m[h, r0 + r, c0 + cc] = (words[r, cc // 32] >> (cc % 32)) & 1
+    return m
+
+
+@pin
+def block_info_hand_built_classes(lib):
+    """Splash-attention mask info (JAX pull request "Support dynamic masks in splash
+    attention"): a block with no attended cell is empty, one with all cells attended is
+    full, any other is partial; the per-row list holds the non-empty blocks in order."""
+    H, Lq, Lk, b = 1, 8, 12, 4
+    m = np.zeros((H, Lq, Lk), np.uint8)
+    m[0, 0:4, 4:8] = 1          # (0,1) full
+    m[0, 1, 9] = 1              # (0,2) partial
+    m[0, 4:8, 0:4] = 1
+    m[0, 6, 2] = 0              # (1,0) partial
+    m[0, 4:8, 8:12] = 1         # (1,2) full
+    info = oracle.block_mask_info(m, b, b, lib=lib)
+    assert info["cls"].tolist() == [[[0, 2, 1], [1, 0, 2]]]
+    assert info["count"].tolist() == [[2, 2]]
+    assert [int(x) for x in info["list"][0, 0, :2]] == [1 | (2 << 30), 2 | (1 << 30)]
+    assert [int(x) for x in info["list"][0, 1, :2]] == [0 | (1 << 30), 2 | (2 << 30)]
+    assert int(info["bits"][0, 0, 2, 1, 0]) == 1 << 1
+    assert int(info["bits"][0, 1, 0, 2, 0]) == 0b1011
+
+
+@pin
+def block_info_round_trip_ragged(lib):
+    """Brute force: on random masks with ragged edges, the classes count the attended cells
+    correctly and the packed partial bits rebuild the mask exactly."""
+    rng = _rng(53)
+    H, Lq, Lk, bq, bk = 2, 37, 70, 16, 32
+    m = (rng.random((H, Lq, Lk)) < 0.5).astype(np.uint8)
+    m[:, :16, :32] = 0
+    m[:, 16:32, 32:64] = 1
+    m[:, 32:37, 64:70] = 1  # a full block at the ragged corner
+    info = oracle.block_mask_info(m, bq, bk, lib=lib)
+    np.testing.assert_array_equal(_decode_info(info, H, Lq, Lk, bq, bk), m)
+    for h in range(H):
+        for qb in range(info["cls"].shape[1]):
+            for kb in range(info["cls"].shape[2]):
+                blk = m[h, qb * bq:(qb + 1) * bq, kb * bk:(kb + 1) * bk]
+                want = 0 if blk.sum() == 0 else (2 if blk.all() else 1)
+                assert info["cls"][h, qb, kb] == want
+            n = info["count"][h, qb]
+            assert n == int((info["cls"][h, qb] != 0).sum())
+            kbs = [int(x) & ((1 << 30) - 1) for x in info["list"][h, qb, :n]]
+            assert kbs == sorted(kbs) and all(info["cls"][h, qb, kb] != 0 for kb in kbs)

@@ -1,0 +1,54 @@
+"""Plausible mistakes planted in copies of the oracle (on the CPU) must each fail a pin.
+
+Each mutant is the oracle's C source with one textual change, compiled into a temporary
+library; the pins of oracle_pins.py then run against it and at least one must fail. This
+shows the pins are strong enough that a dropped term, a wrong sign, index or operand in the
+oracle would not go unnoticed.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "sdpa_oracle.c")
+
+MUTANTS = {
+    "causal_off_by_one": ("!(j <= off + i)", "!(j < off + i)"),
+    "gqa_interleaved_heads": ("? (h / group) :", "? (h % Hkv) :"),
+    "bottom_right_sign": ("off = kvlen_b - qlen_b;", "off = qlen_b - kvlen_b;"),
+    "scale_dropped": ("double x = scale * dot;", "double x = dot;"),
+    "kv_length_inclusive": ("int ok = (j < kvlen_b);", "int ok = (j <= kvlen_b);"),
+    "q_length_inclusive": ("if (i >= qlen_b) {", "if (i > qlen_b) {"),
+    "mask_strides_swapped": ("p->mask[j * p->mask_stride[0] + i * p->mask_stride[1]",
+                             "p->mask[i * p->mask_stride[0] + j * p->mask_stride[1]"),
+    "bias_sign": ("      x += p->bias[", "      x -= p->bias["),
+    "bias_scaled": ("    s[j] = x;\n", "    s[j] = x * 0.5 + 0.5 * scale * dot;\n"),
+    "not_normalised": ("const double w = s[j] / denom;", "const double w = s[j];"),
+    "empty_row_zero": ("o[e] = NAN;", "o[e] = 0.0;"),
+    "default_scale_dv": ("1.0 / sqrt((double)D)", "1.0 / sqrt((double)Dv)"),
+    "value_head_wrong": ("const double* vj = v + ((b * Lk + j) * Hkv + g) * Dv;",
+                         "const double* vj = v + ((b * Lk + j) * Hkv + (g + 1) % Hkv) * Dv;"),
+    "cache_rows_reversed": ("index[b] + t) * row", "index[b] + n_new - 1 - t) * row"),
+    "block_class_swapped": ("(set == cells ? 2 : 1)", "(set == cells ? 1 : 2)"),
+    "block_bits_reversed": ("word |= (1u << c);", "word |= (1u << (31 - c));"),
+    "block_full_at_edge": ("(set == cells ? 2 : 1)", "(set == bq * bk ? 2 : 1)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_fails_a_pin(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new, 1))
+    lib = oracle.load(oracle.build(str(mutated), str(tmp_path / "libmutant.so"), force=True))
+    failed = []
+    for p in PINS:
+        try:
+            p(lib)
+        except Exception as e:  # noqa: BLE001 — any failure counts
+            failed.append(p.__name__)
+    assert failed, f"mutant {name} passed every pin"
