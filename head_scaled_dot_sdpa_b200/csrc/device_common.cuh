@@ -1,0 +1,98 @@
+// Device helpers shared by the kernels: element conversion, status reporting and the
+// per-batch resolution of lengths and causal offsets.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "internal.h"
+
+namespace sdpa {
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Records the first device-side error in the status word; later errors keep the first.
+__device__ __forceinline__ void report(int* status, int code) {
+  if (status) atomicCAS(status, kStatusOk, code);
+}
+
+// Lengths, offsets: the arguments q_lengths, kv_lengths, q_offset and is_causal of
+// NNlib.scaled_dot_product_attention. Out-of-range lengths are clamped and reported.
+__device__ __forceinline__ BatchInfo resolve_batch(const Problem& P, int b) {
+  BatchInfo bi;
+  bi.skip = false;
+  int ql = P.Lq, kl = P.Lk;
+  if (P.q_lengths) {
+    ql = P.q_lengths[b];
+    if (ql < 0 || ql > P.Lq) {
+      report(P.status, SDPA_ERR_DEVICE_CHECK);
+      ql = ql < 0 ? 0 : P.Lq;
+    }
+  }
+  if (P.cache_index) {
+    const int idx = P.cache_index[b];
+    bi.skip = idx < 0 || idx > P.Lk - P.Lq;  // reported by the cache update
+    kl = bi.skip ? 0 : idx + P.Lq;
+  } else if (P.kv_lengths) {
+    kl = P.kv_lengths[b];
+  }
+  if (kl < 0 || kl > P.Lk) {
+    report(P.status, SDPA_ERR_DEVICE_CHECK);
+    kl = kl < 0 ? 0 : P.Lk;
+  }
+  bi.q_len = ql;
+  bi.kv_len = kl;
+  if (P.causal == SDPA_CAUSAL_TOP_LEFT)
+    bi.offset = P.q_offset ? P.q_offset[b] : P.q_offset_scalar;
+  else if (P.causal == SDPA_CAUSAL_BOTTOM_RIGHT)
+    bi.offset = kl - ql;
+  else
+    bi.offset = 0x3fffffff;  // no causal limit
+  return bi;
+}
+
+// Bias element (key j, query i, head h, batch b), as float.
+__device__ __forceinline__ float load_bias(const Problem& P, int b, int h, long long i,
+                                           long long j) {
+  const long long off = j * P.bs[0] + i * P.bs[1] + (long long)h * P.bs[2] + (long long)b * P.bs[3];
+  switch (P.bias_dtype) {
+    case SDPA_F16: return __half2float(static_cast<const __half*>(P.bias)[off]);
+    case SDPA_BF16: return __bfloat162float(static_cast<const __nv_bfloat16*>(P.bias)[off]);
+    default: return static_cast<const float*>(P.bias)[off];
+  }
+}
+
+// Whether the boolean mask (dense, or its block classification) lets query i of head h see
+// key j. The block classification, when present, takes precedence over the dense mask.
+__device__ __forceinline__ bool mask_allows(const Problem& P, int b, int h, int i, int j) {
+  if (P.bcls) {
+    const int hm = P.bi_nheads == 1 ? 0 : h;
+    const int qb = i / P.bi_bq, kb = j / P.bi_bk;
+    const long long blk = ((long long)hm * P.bi_nqb + qb) * P.bi_nkb + kb;
+    const uint8_t c = P.bcls[blk];
+    if (c == SDPA_BLOCK_EMPTY) return false;
+    if (c == SDPA_BLOCK_FULL) return true;
+    const int words = P.bi_bk / 32;
+    const int r = i - qb * P.bi_bq, cc = j - kb * P.bi_bk;
+    const uint32_t w = P.bbits[(blk * P.bi_bq + r) * words + cc / 32];
+    return (w >> (cc % 32)) & 1u;
+  }
+  if (P.mask) {
+    const long long off = (long long)j * P.ms[0] + (long long)i * P.ms[1] +
+                          (long long)h * P.ms[2] + (long long)b * P.ms[3];
+    return P.mask[off] != 0;
+  }
+  return true;
+}
+
+}  // namespace sdpa

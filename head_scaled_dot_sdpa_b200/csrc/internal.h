@@ -1,0 +1,73 @@
+// Internal declarations shared by the host resolver (sdpa_api.cu) and the kernels.
+// Nothing here is part of the public ABI in include/sdpa.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/sdpa.h"
+
+namespace sdpa {
+
+// Status word values written by kernels (first error wins, via atomicCAS from SDPA_OK).
+constexpr int kStatusOk = SDPA_OK;
+
+// A call with every host-side argument resolved and validated. Per-batch values that live on
+// the device (lengths, offsets, cache indices) stay there and are resolved by the kernels.
+struct Problem {
+  int dtype;                 // sdpa_dtype of q/k/v/out
+  int B, Lq, Lk, H, Hkv, D, Dv, group;
+  float scale;               // resolved (1/sqrt(D) when NaN was given)
+  float scale_log2;          // scale * log2(e)
+  int causal;                // sdpa_causal
+  int q_offset_scalar;
+  const int32_t* q_offset;   // device [B] or null
+  const int32_t* q_lengths;  // device [B] or null
+  const int32_t* kv_lengths; // device [B] or null
+  const int32_t* cache_index;  // decode: kv_len[b] = cache_index[b] + Lq; else null
+  const void* bias;
+  int bias_dtype;
+  long long bs[4];           // bias strides (j, i, h, b) in elements
+  const uint8_t* mask;
+  long long ms[4];           // mask strides (j, i, h, b)
+  // block info (null bcls when absent)
+  const uint8_t* bcls;
+  const int32_t* brow_count;
+  const uint32_t* brow_list;
+  const uint32_t* bbits;
+  int bi_nheads, bi_nqb, bi_nkb, bi_bq, bi_bk;
+  int* status;               // device status word (never null when a kernel runs)
+};
+
+// Per-batch values every kernel resolves the same way.
+struct BatchInfo {
+  int q_len;   // valid queries
+  int kv_len;  // valid keys
+  int offset;  // causal offset (query i attends keys j <= offset + i)
+  bool skip;   // decode: the cache index is out of range, leave this sequence alone
+};
+
+// Launchers (each returns a cudaError_t from the launch).
+cudaError_t launch_generic(const Problem& P, const void* q, const void* k, const void* v,
+                           void* out, cudaStream_t stream);
+cudaError_t launch_cache_update(void* k_cache, void* v_cache, const void* k_new,
+                                const void* v_new, int esize, int d, int Hkv, int n_new,
+                                int capacity, int B, const int32_t* index, int* status,
+                                cudaStream_t stream);
+size_t decode_workspace_bytes(const Problem& P);
+bool decode_supported(const Problem& P);
+cudaError_t launch_decode(const Problem& P, const void* q, const void* k_cache,
+                          const void* v_cache, void* out, void* ws_partials,
+                          cudaStream_t stream);
+cudaError_t launch_block_classify(const uint8_t* mask, const long long ms[3], int H, int Lq,
+                                  int Lk, int bq, int bk, uint8_t* cls, int32_t* count,
+                                  uint32_t* list, uint32_t* bits, int* status,
+                                  cudaStream_t stream);
+bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v,
+                       const void* out);
+size_t prefill_workspace_bytes(const Problem& P);
+cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const void* v,
+                           void* out, void* ws_sched, cudaStream_t stream,
+                           const char** error_message);
+
+}  // namespace sdpa

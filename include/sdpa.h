@@ -1,0 +1,209 @@
+/*
+ * sdpa.h — C ABI of libsdpa.so: the forward pass of multi-head scaled-dot-product attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation is NNlib.scaled_dot_product_attention as the Flux.jl page "Neural Network
+ * primitives from NNlib.jl" defines it (entry "scaled_dot_product_attention", section
+ * "Arguments"):
+ *
+ *     out = softmax(scale * query' * key + bias, masked) * value
+ *
+ * with grouped-query sharing of key/value heads, is_causal (top-left with q_offset, or
+ * :bottom_right), per-batch q_lengths / kv_lengths, a broadcast additive bias and a boolean
+ * mask, computed tile by tile with an online softmax (section "Fused implementation").
+ *
+ * Conventions for every call:
+ *  - Layout. q, k, v and out are dense arrays in the page's column-major
+ *    (head_dim, nheads, seq_len, batch) order, which is row-major [batch][seq][head][dim]:
+ *      q   [batch][q_len ][nheads  ][dqk]
+ *      k   [batch][kv_len][nkvheads][dqk]
+ *      v   [batch][kv_len][nkvheads][dv ]
+ *      out [batch][q_len ][nheads  ][dv ]
+ *    Several trailing batch dimensions of the page are flattened into one `batch`.
+ *  - Ownership. Every data pointer is a DEVICE pointer owned by the caller; the library keeps
+ *    no reference after the call returns and allocates no device memory. Scratch space is a
+ *    caller-owned workspace sized by sdpa_workspace_size().
+ *  - Asynchrony. Calls enqueue work on `stream` and return without synchronising. Lengths and
+ *    offsets that live on the device are never read on the host.
+ *  - Errors. Invalid arguments are reported before anything is launched, as a status code;
+ *    sdpa_last_error() gives a message. Errors found on the device (an out-of-range cache
+ *    index, a bounded wait that ran out) are recorded in the workspace's status word and read
+ *    with sdpa_read_device_status(). No call aborts the process or traps the GPU.
+ */
+#ifndef SDPA_H_
+#define SDPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t */
+
+#if defined(__GNUC__)
+#define SDPA_API __attribute__((visibility("default")))
+#else
+#define SDPA_API
+#endif
+
+typedef enum {
+  SDPA_OK = 0,
+  SDPA_ERR_INVALID_ARG = 1, /* shape, stride, pointer or enum out of range */
+  SDPA_ERR_UNSUPPORTED = 2, /* valid request that no kernel here implements */
+  SDPA_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+  SDPA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  SDPA_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out (read via the status word) */
+  SDPA_ERR_DEVICE_CHECK = 6 /* device: an index check failed, the access was skipped */
+} sdpa_status;
+
+typedef enum { SDPA_F32 = 0, SDPA_F16 = 1, SDPA_BF16 = 2 } sdpa_dtype;
+
+/* Argument is_causal: false, true (query i attends keys j <= q_offset + i), or :bottom_right
+ * (q_offset = kv_lengths - q_lengths, the array sizes standing in for lengths not given). */
+typedef enum {
+  SDPA_CAUSAL_NONE = 0,
+  SDPA_CAUSAL_TOP_LEFT = 1,
+  SDPA_CAUSAL_BOTTOM_RIGHT = 2
+} sdpa_causal;
+
+/* Block classes of a boolean mask (splash-attention mask info of the JAX pull request
+ * "Support dynamic masks in splash attention"; this encoding is this library's own). */
+enum { SDPA_BLOCK_EMPTY = 0, SDPA_BLOCK_PARTIAL = 1, SDPA_BLOCK_FULL = 2 };
+
+/* Result of build_block_mask_info(); every pointer is into the caller's info buffer.
+ *  block_class [nheads][nqb][nkb]     SDPA_BLOCK_* of each bq x bk block
+ *  row_count   [nheads][nqb]          number of non-empty blocks in block row qb
+ *  row_list    [nheads][nqb][nkb]     the first row_count entries: kb | (class << 30), kb
+ *                                     increasing
+ *  partial_bits[nheads][nqb][nkb][bq][bk/32]  for PARTIAL blocks only: bit c of word w of
+ *                                     row r is mask(head, qb*bq + r, kb*bk + 32*w + c);
+ *                                     cells past q_len / kv_len are 0.
+ * nheads is the mask's own head extent (1 when it is broadcast over heads). */
+typedef struct sdpa_block_mask_info {
+  int32_t nheads, q_len, kv_len, bq, bk, nqb, nkb;
+  const uint8_t* block_class;
+  const int32_t* row_count;
+  const uint32_t* row_list;
+  const uint32_t* partial_bits;
+} sdpa_block_mask_info;
+
+/* Flags (sdpa_params.flags). */
+#define SDPA_FLAG_GENERIC_KERNEL 0x1u /* force the SIMT kernel (any dtype / head size) */
+
+/* One attention call. Arguments of the page's entry and where they sit here:
+ *  dtype            element type of q, k, v and out (fp32 accumulation throughout; out is
+ *                   rounded to nearest even).
+ *  batch, q_len, kv_len, nheads, nkvheads, dqk, dv   the array sizes. nheads % nkvheads must
+ *                   be 0 (GQA paragraph); query head h uses key/value head
+ *                   h / (nheads / nkvheads).
+ *  scale            multiplier of query'*key; NaN means 1/sqrt(dqk) (argument `scale`).
+ *  causal, q_offset_scalar, q_offset   argument `is_causal` and `q_offset`: q_offset is a
+ *                   device int32[batch] or NULL for q_offset_scalar; ignored unless
+ *                   causal == SDPA_CAUSAL_TOP_LEFT.
+ *  q_lengths, kv_lengths   device int32[batch] or NULL (full length). Keys j >= kv_lengths[b]
+ *                   are not attended; output rows i >= q_lengths[b] are zero. Values must
+ *                   lie in [0, q_len] / [0, kv_len].
+ *  bias             NULL or a device array of bias_dtype, element (key j, query i, head h,
+ *                   batch b) at bias[j*bias_stride[0] + i*bias_stride[1] + h*bias_stride[2]
+ *                   + b*bias_stride[3]]; a stride of 0 broadcasts (argument `bias`: added to
+ *                   the logits, not scaled).
+ *  mask             NULL or a device uint8 array (0 = not attended), addressed like the bias
+ *                   with mask_stride (argument `mask`). mask, is_causal and kv_lengths
+ *                   combine by AND.
+ *  block_info       NULL, or the classification of `mask` built by build_block_mask_info;
+ *                   then empty blocks are skipped and only partial blocks' bits are read
+ *                   (`mask` may then be NULL). The mask it describes must not vary with batch.
+ *  flags            SDPA_FLAG_* bits. */
+typedef struct sdpa_params {
+  sdpa_dtype dtype;
+  int32_t batch, q_len, kv_len, nheads, nkvheads, dqk, dv;
+  float scale;
+  sdpa_causal causal;
+  int32_t q_offset_scalar;
+  const int32_t* q_offset;
+  const int32_t* q_lengths;
+  const int32_t* kv_lengths;
+  const void* bias;
+  sdpa_dtype bias_dtype;
+  int64_t bias_stride[4];
+  const uint8_t* mask;
+  int64_t mask_stride[4];
+  const sdpa_block_mask_info* block_info;
+  uint32_t flags;
+} sdpa_params;
+
+/* Bytes of workspace sdpa_forward / sdpa_decode_with_cache need for these params (at least
+ * 256: the device status word lives at the start). The workspace must be 256-byte aligned.
+ * Returns 0 if the params are invalid. */
+SDPA_API size_t sdpa_workspace_size(const sdpa_params* p);
+
+/* Writes the status word at the start of `ws` to SDPA_OK (enqueued on `stream`). Call once on
+ * a fresh workspace before the first use; kernels only ever set it to an error. */
+SDPA_API sdpa_status sdpa_workspace_init(void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* scaled_dot_product_attention(q, k, v, [bias]; mask, scale, is_causal, q_offset, q_lengths,
+ * kv_lengths) into `out` (device, caller-owned, same dtype as q). A query attending to no key
+ * gives NaN (section "Fused implementation"). Returns SDPA_OK once the work is enqueued. */
+SDPA_API sdpa_status sdpa_forward(const sdpa_params* p, const void* q, const void* k, const void* v,
+                         void* out, void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* Decoding with a KV cache (the page's example "decoding with a KV cache"; the Keras issue
+ * "MultiHeadAttention is missing a position_bias call argument", cache_update_index):
+ * writes k_new/v_new [batch][n_new][nkvheads][d] into k_cache/v_cache
+ * [batch][capacity][nkvheads][d] at rows cache_index[b] .. cache_index[b] + n_new - 1, then
+ * attends the n_new queries q [batch][n_new][nheads][dqk] with is_causal=:bottom_right and
+ * kv_lengths[b] = cache_index[b] + n_new. Here p->q_len = n_new, p->kv_len = capacity,
+ * p->causal must be SDPA_CAUSAL_BOTTOM_RIGHT and q_lengths, kv_lengths, bias, mask and
+ * block_info must be NULL. cache_index is a device int32[batch]; a value outside
+ * [0, capacity - n_new] skips that sequence's write and attention (its output rows are left
+ * as they were) and sets SDPA_ERR_DEVICE_CHECK in the status word. */
+SDPA_API sdpa_status sdpa_decode_with_cache(const sdpa_params* p, const void* q, const void* k_new,
+                                   const void* v_new, void* k_cache, void* v_cache,
+                                   const int32_t* cache_index, void* out, void* ws,
+                                   size_t ws_bytes, struct CUstream_st* stream);
+
+/* Writes k_new/v_new [batch][n_new][nkvheads][d] of `dtype` into the caches
+ * [batch][capacity][nkvheads][d] at rows index[b] + t, t < n_new (index: device
+ * int32[batch]). Either cache pair may be NULL to update only the other. An index outside
+ * [0, capacity - n_new] skips that sequence and sets SDPA_ERR_DEVICE_CHECK in the status word
+ * of `ws` (ws may be NULL, in which case the check is silent). */
+SDPA_API sdpa_status cache_update_at_index(void* k_cache, void* v_cache, const void* k_new,
+                                  const void* v_new, sdpa_dtype dtype, int32_t d,
+                                  int32_t nkvheads, int32_t n_new, int32_t capacity,
+                                  int32_t batch, const int32_t* index, void* ws,
+                                  struct CUstream_st* stream);
+
+/* Bytes of info buffer build_block_mask_info needs (256-byte aligned). bk must be a multiple
+ * of 32. Returns 0 if the sizes are invalid. */
+SDPA_API size_t build_block_mask_info_size(int32_t nheads, int32_t q_len, int32_t kv_len, int32_t bq,
+                                  int32_t bk);
+
+/* Classifies every bq x bk block of a boolean mask (device uint8, element (key j, query i,
+ * head h) at mask[j*mask_stride[0] + i*mask_stride[1] + h*mask_stride[2]]; mask_stride[0]
+ * must be 1) as empty, partial or full, packs the bits of the partial blocks and lists the
+ * non-empty blocks of every block row (see sdpa_block_mask_info). The result lives in the
+ * caller's `info_buf` and is described by *out_info, filled in on the host before return.
+ * sdpa_forward uses it when bq = bk = 128. */
+SDPA_API sdpa_status build_block_mask_info(const uint8_t* mask, const int64_t mask_stride[3],
+                                  int32_t nheads, int32_t q_len, int32_t kv_len, int32_t bq,
+                                  int32_t bk, void* info_buf, size_t info_bytes,
+                                  sdpa_block_mask_info* out_info, struct CUstream_st* stream);
+
+/* Synchronises `stream`, returns the status word of `ws` (SDPA_OK or the first device error)
+ * and resets it to SDPA_OK. For tests and diagnostics; not for the hot path. */
+SDPA_API sdpa_status sdpa_read_device_status(void* ws, struct CUstream_st* stream);
+
+/* Message for the last non-OK status returned on this host thread. */
+SDPA_API const char* sdpa_last_error(void);
+
+/* Name of the kernel the last sdpa_forward / sdpa_decode_with_cache call on this host thread
+ * launched for its attention ("generic_simt", "prefill_tcgen05", "decode_splitkv"). */
+SDPA_API const char* sdpa_last_kernel(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_H_ */
