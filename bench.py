@@ -1,0 +1,421 @@
+"""Benchmark of the attention hot path on B200; prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline: causal GQA prefill (batch 4, 32 query / 8 key-value heads, head_dim 128, 2048
+queries and keys, bf16, fp32 accumulation), TFLOP/s over the unmasked (attended) pairs,
+4*head_dim flops per pair. The same line carries the other workloads of the hot path, each
+timed the same way: KV-cache decode (HBM GB/s), ALiBi/T5 bias attention (fp16), and
+block-sparse masked attention (with its block classification pass).
+
+Timing: W untimed warm-up steps, then K steps, each preceded by an L2 flush (a 256 MiB write)
+and timed on the launching stream with CUDA events; the K steps are bracketed by a barrier and
+torch.cuda.synchronize() and the max over ranks is taken. With N GPUs every rank runs its own
+copy of the workload (independent batches; no collective on the data path): weak scaling.
+
+--impl reference times the CPU float64 oracle (the slow reference program) on a bounded
+sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import sdpa_inputs as si  # noqa: E402
+
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def causal_pairs(Lq, Lk, offset=0):
+    """Number of (query, key) pairs with key <= offset + query, key < Lk."""
+    i = np.arange(Lq, dtype=np.int64)
+    return int(np.clip(offset + i + 1, 0, Lk).sum())
+
+
+# ---- distributed plumbing -------------------------------------------------------------------
+
+def init_dist(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- clocks ---------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---- timing ---------------------------------------------------------------------------------
+
+def time_steps(step, steps, warmup, world, stream=None):
+    """Device time (ms) of each of `steps` calls of step(), each after an L2 flush."""
+    stream = stream or torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for s in range(steps):
+        flush.zero_()
+        starts[s].record(stream)
+        step()
+        ends[s].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    per = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    return per
+
+
+# ---- workloads --------------------------------------------------------------------------------
+
+def prefill_case(dev):
+    w = si.CAUSAL_GQA_PREFILL
+    q, k, v = si.qkv(w)
+    flops = 4.0 * w.head_dim * w.batch * w.nheads * causal_pairs(w.q_len, w.kv_len)
+    byts = (q.numel() + k.numel() + v.numel() + q.numel()) * 2
+    return w, (q, k, v), flops, byts
+
+
+def run_ours(args, rank, world, local):
+    import head_scaled_dot_sdpa_b200 as sdpa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = _peaks()
+    stream = torch.cuda.current_stream()
+    result = {}
+
+    # ---- headline: causal GQA prefill
+    w, (q, k, v), flops, byts = prefill_case(dev)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty_like(qd)
+    ws = sdpa.Workspace(dev)
+    step = lambda: sdpa.sdpa_forward(qd, kd, vd, is_causal=True, out=out, workspace=ws)
+    step()
+    kernel = sdpa.last_kernel()
+    with ClockSampler(local) as clk:
+        per = time_steps(step, args.steps, args.warmup, world)
+    ms = max_over_ranks(float(np.sum(per)), world) / args.steps
+    status = sdpa.read_device_status(ws)
+    value = flops * world / (ms * 1e-3) / 1e12
+    kernel_tflops = flops / (float(np.mean(per)) * 1e-3) / 1e12
+
+    # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        sdpa.sdpa_forward(qd, kd, vd, is_causal=True, out=out, workspace=ws)
+        oh.copy_(out, non_blocking=True)
+
+    per_e2e = time_steps(e2e_step, args.steps, args.warmup, world)
+    ms_e2e = max_over_ranks(float(np.sum(per_e2e)), world) / args.steps
+    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
+    d2h = out.numel() * out.element_size()
+
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get("prefill_tcgen05", None)
+
+    result.update({
+        "metric": "prefill attention TFLOP/s (unmasked FLOPs)",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), numpy PCG64)",
+        "config": {"workload": w.name, "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
+                   "nheads": w.nheads, "nkvheads": w.nkvheads, "head_dim": w.head_dim,
+                   "is_causal": True, "flops_per_step": flops,
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replica per GPU x{world} (independent batches)"},
+        "kernel": kernel,
+        "device_status": int(status),
+        "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2), "peak": peaks["bf16"],
+                     "unit": "TFLOP/s", "frac": round(kernel_tflops / peaks["bf16"], 4),
+                     "traffic": traffic, "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": round(kernel_tflops / peaks["bf16_sustained"], 4)},
+        "e2e": {"value": round(flops * world / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    })
+    del qd, kd, vd, out, qh, kh, vh, oh
+
+    if not args.headline_only:
+        result["other_workloads"] = other_workloads(args, dev, world, ws, peaks)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    return result
+
+
+def other_workloads(args, dev, world, ws, peaks):
+    import head_scaled_dot_sdpa_b200 as sdpa
+
+    res = {}
+    # KV-cache decode: HBM GB/s over the bytes a step must move
+    w = si.KV_CACHE_DECODE
+    d = si.decode_inputs(w)
+    qd, kn, vn = d["q"].to(dev), d["k_new"].to(dev), d["v_new"].to(dev)
+    kc, vc = d["k_cache"].to(dev), d["v_cache"].to(dev)
+    idx = d["index"].to(dev)
+    out = torch.empty_like(qd)
+    kl = d["kv_lengths"].numpy().astype(np.int64)
+    byts = (int(kl.sum()) * w.nkvheads * w.head_dim * 2 * 2 + 2 * qd.numel() * 2 + 4 * kn.numel() * 2)
+    step = lambda: sdpa.sdpa_decode_with_cache(qd, kn, vn, kc, vc, idx, out=out, workspace=ws)
+    per = time_steps(step, args.steps, args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    gbs = byts / (ms * 1e-3) / 1e9
+    res["kv_cache_decode"] = {"workload": w.name, "metric": "decode HBM GB/s", "value": round(gbs * world, 1),
+                              "unit": "GB/s", "ms_per_step": round(ms, 4), "bytes_per_step": byts,
+                              "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"],
+                                           "unit": "GB/s", "frac": round(gbs / peaks["hbm"], 4)},
+                              "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 4}
+    del qd, kn, vn, kc, vc, out
+
+    # ALiBi/T5 bias attention
+    w = si.ALIBI_T5_BIAS
+    q, k, v = [t.to(dev) for t in si.qkv(w)]
+    bias = si.alibi_t5_bias(w).to(dev)
+    out = torch.empty_like(q)
+    flops = 4.0 * w.head_dim * w.batch * w.nheads * causal_pairs(w.q_len, w.kv_len)
+    step = lambda: sdpa.sdpa_forward(q, k, v, bias, is_causal=True, out=out, workspace=ws)
+    per = time_steps(step, args.steps, args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    bias_bytes = w.nheads * causal_pairs(w.q_len, w.kv_len) * 2
+    res["alibi_t5_bias"] = {"workload": w.name, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2),
+                            "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+                            "bias_GBs": round(bias_bytes / (ms * 1e-3) / 1e9, 1), "kernel": sdpa.last_kernel()}
+    del q, k, v, bias, out
+
+    # block-sparse mask: classification pass + attention over the non-empty blocks
+    w = si.BLOCK_SPARSE
+    cls = si.block_classes(w)
+    mask = si.mask_device(w, cls, dev)
+    allowed = int(mask.sum(dtype=torch.int64).item())
+    q, k, v = [t.to(dev) for t in si.qkv(w)]
+    out = torch.empty_like(q)
+    info = sdpa.build_block_mask_info(mask)
+    step_c = lambda: sdpa.build_block_mask_info(mask)
+    per_c = time_steps(step_c, args.steps, args.warmup, world)
+    ms_c = max_over_ranks(float(np.mean(per_c)), world)
+    step = lambda: sdpa.sdpa_forward(q, k, v, block_info=info, out=out, workspace=ws)
+    per = time_steps(step, args.steps, args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    flops = 4.0 * w.head_dim * allowed
+    n_blocks = int((cls != 0).sum())
+    res["block_sparse_mask"] = {
+        "workload": w.name, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2), "unit": "TFLOP/s (unmasked)",
+        "ms_per_step": round(ms, 4), "executed_tflops": round(4.0 * w.head_dim * n_blocks * 128 * 128 / (ms * 1e-3) / 1e12, 2),
+        "classification": {"ms": round(ms_c, 4), "GB/s": round(mask.numel() / (ms_c * 1e-3) / 1e9, 1),
+                           "frac_hbm": round(mask.numel() / (ms_c * 1e-3) / 1e9 / peaks["hbm"], 4)},
+        "kernel": sdpa.last_kernel()}
+    return res
+
+
+# ---- CPU oracle ---------------------------------------------------------------------------------
+
+def _oracle_heads(q, k, v, heads, group):
+    """Run the oracle on (b, h) heads of the causal GQA workload, one head per call."""
+    import oracle
+    qn, kn, vn = (t.float().numpy() for t in (q, k, v))
+    flops = 0.0
+    for b, h in heads:
+        g = h // group
+        oracle.sdpa_forward(qn[b:b + 1, :, h:h + 1], kn[b:b + 1, :, g:g + 1], vn[b:b + 1, :, g:g + 1],
+                            is_causal=True)
+        flops += 4.0 * q.shape[3] * causal_pairs(q.shape[1], k.shape[1])
+    return flops
+
+
+def cpu_baseline(budget_s=20.0):
+    import oracle
+    oracle.load()
+    w = si.CAUSAL_GQA_PREFILL
+    q, k, v = si.qkv(w)
+    group = w.nheads // w.nkvheads
+    all_heads = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
+    t0 = time.perf_counter()
+    flops, done = 0.0, 0
+    for chunk in range(0, len(all_heads), 8):
+        flops += _oracle_heads(q, k, v, all_heads[chunk:chunk + 8], group)
+        done += len(all_heads[chunk:chunk + 8])
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"{done} of {len(all_heads)} (batch, head) rows of the causal GQA workload, float64, "
+                      f"{dt:.1f} s wall"}
+
+
+def run_reference(args, rank, world):
+    """The slow reference program: the CPU oracle, timed per step on a bounded sample."""
+    import oracle
+    oracle.load()
+    w = si.CAUSAL_GQA_PREFILL
+    q, k, v = si.qkv(w)
+    group = w.nheads // w.nkvheads
+    heads = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
+    per_step = max(1, args.reference_heads)
+    for s in range(args.warmup):
+        _oracle_heads(q, k, v, heads[:per_step], group)
+    times, flops = [], 0.0
+    for s in range(args.steps):
+        sel = [heads[(s * per_step + j) % len(heads)] for j in range(per_step)]
+        t0 = time.perf_counter()
+        flops = _oracle_heads(q, k, v, sel, group)
+        times.append(time.perf_counter() - t0)
+    ms = float(np.mean(times)) * 1e3
+    value = flops / (ms * 1e-3) / 1e12
+    return {
+        "impl": "reference",
+        "metric": "prefill attention TFLOP/s (unmasked FLOPs)",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), numpy PCG64)",
+        "config": {"workload": w.name, "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
+                   "nheads": w.nheads, "nkvheads": w.nkvheads, "head_dim": w.head_dim, "is_causal": True,
+                   "step": f"{per_step} (batch, head) rows of the workload per step"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                         "kind": "oracle", "sample": f"{per_step} (batch, head) rows per step, float64"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--reference-heads", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+
+    rank, world, local = init_dist(args.gpus)
+    try:
+        res = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

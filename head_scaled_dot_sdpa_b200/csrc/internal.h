@@ -37,6 +37,7 @@ struct Problem {
   const uint32_t* bbits;
   int bi_nheads, bi_nqb, bi_nkb, bi_bq, bi_bk;
   int* status;               // device status word (never null when a kernel runs)
+  unsigned long long wait_timeout_ns;  // bound on every mbarrier wait of the tcgen05 kernel
 };
 
 // Per-batch values every kernel resolves the same way.

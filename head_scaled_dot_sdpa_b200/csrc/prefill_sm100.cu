@@ -1,16 +1,104 @@
-// Placeholder until the tcgen05 prefill kernel lands: every call takes the SIMT kernel.
-#include "internal.h"
+// Host side of the tcgen05 prefill kernel (prefill_sm100.cuh): which calls it takes, the TMA
+// tensor maps of Q, K and V, and the launch of the bias / mask variant the call needs.
+#include <algorithm>
+
+#include "prefill_sm100.cuh"
 
 namespace sdpa {
+namespace {
 
-bool prefill_supported(const Problem&, const void*, const void*, const void*, const void*) {
-  return false;
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up at run time (the library does not link libcuda).
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
 }
+
+// A (batch, seq, heads, dim) array as a 4-d tensor map; box = 64 dims x 128 rows, 128B swizzle
+// (the K-major / MN-major operand layout the MMA descriptors assume). Rows past `seq` read 0.
+bool make_map(CUtensorMap* m, const void* base, int dtype, int D, int heads, int seq, int batch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)seq, (cuuint64_t)batch};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2, (cuuint64_t)seq * heads * D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt = dtype == SDPA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = [] {
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v > 0 ? v : 148;
+  }();
+  return n;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out) {
+  if (P.dtype != SDPA_BF16 && P.dtype != SDPA_F16) return false;
+  if (P.D != P.Dv || (P.D != 64 && P.D != 128)) return false;
+  if (P.Lq <= 0 || P.Lk <= 0 || P.B <= 0) return false;
+  if (!(P.scale > 0.f)) return false;  // the row max is taken on scaled logits
+  if (P.bcls && (P.bi_bq != prefill::kBlockM || P.bi_bk != prefill::kBlockN)) return false;
+  if ((long long)P.B * P.H * ((P.Lq + 127) / 128) >= (1LL << 30)) return false;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return false;
+  if (P.bias) {
+    // contiguous along keys, 16-byte aligned rows; the bias type is the input type or fp32
+    const int es = P.bias_dtype == SDPA_F32 ? 4 : 2;
+    if (P.bias_dtype != SDPA_F32 && P.bias_dtype != P.dtype) return false;
+    if (P.bs[0] != 1 || !aligned(P.bias, 16)) return false;
+    for (int d = 1; d < 4; ++d)
+      if ((P.bs[d] * es) % 16 != 0) return false;
+  }
+  if (P.mask && !P.bcls) {
+    if (P.ms[0] != 1 || !aligned(P.mask, 16)) return false;
+    for (int d = 1; d < 4; ++d)
+      if (P.ms[d] % 16 != 0) return false;
+  }
+  return encode_fn() != nullptr;
+}
+
 size_t prefill_workspace_bytes(const Problem&) { return 0; }
-cudaError_t launch_prefill(const Problem&, const void*, const void*, const void*, void*, void*,
-                           cudaStream_t, const char** msg) {
-  if (msg) *msg = "prefill kernel not built";
-  return cudaErrorNotSupported;
+
+cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const void* v, void* out, void*,
+                           cudaStream_t stream, const char** msg) {
+  prefill::TensorMaps maps;
+  if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
+      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B)) {
+    if (msg) *msg = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
+  const int grid = (int)std::min<long long>(n_units, sm_count());
+  cudaError_t e;
+  if (P.dtype == SDPA_BF16)
+    e = P.D == 128 ? prefill::launch<__nv_bfloat16, 128>(maps, P, out, grid, stream)
+                   : prefill::launch<__nv_bfloat16, 64>(maps, P, out, grid, stream);
+  else
+    e = P.D == 128 ? prefill::launch<__half, 128>(maps, P, out, grid, stream)
+                   : prefill::launch<__half, 64>(maps, P, out, grid, stream);
+  if (e != cudaSuccess && msg) *msg = "prefill launch";
+  return e;
 }
 
 }  // namespace sdpa

@@ -1,0 +1,688 @@
+// Tiled online-softmax attention for sm_100a (B200): the fused implementation of
+// NNlib.scaled_dot_product_attention (Flux.jl page "Neural Network primitives from NNlib.jl",
+// section "Fused implementation": tile by tile, online softmax over key tiles, weights never
+// materialised), for fp16/bf16 inputs with qk_head_dim = v_head_dim in {64, 128}.
+//
+// Work unit: two 128-query tiles A and B that read the same key/value head of the same batch
+// element: two query heads of one GQA group (same query tile), or, without GQA, two adjacent
+// query tiles of one head. Persistent CTAs (one per SM) walk the units, longest causal rows
+// first. The key tiles a unit visits are the union of the two tiles' lists (the causal /
+// kv_lengths prefix, or the non-empty blocks of a block-sparse mask), each loaded once.
+//
+// Warp roles (384 threads):
+//   warp 8      TMA producer: Q_A, Q_B, then K_u ahead of V_{u-1} through 128B-swizzled rings;
+//   warp 9      MMA issuer and TMEM owner (warps 10-11 idle; warpgroup 2 gives its registers to
+//               the softmax warpgroups with setmaxnreg). Per key tile u, in this order:
+//                 O_A += P_A(u-1) V(u-1);  S_A(u) = Q_A K(u)^T;
+//                 O_B += P_B(u-1) V(u-1);  S_B(u) = Q_B K(u)^T
+//               (S: tcgen05.mma with both operands in shared memory; PV: P read from TMEM). So
+//               the tensor pipe works on one tile while the other tile's softmax runs, and the
+//               in-order tcgen05 pipeline lets S_X(u) reuse the columns PV_X(u-1) just read;
+//   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: one thread per query row
+//               (= TMEM lane). tcgen05.ld of the S row; masks (causal / q_offset / kv_lengths
+//               as one prefix bound per row, boolean mask bytes or partial-block bits); optional
+//               bias; row max; P = 2^(s*scale*log2e - m) written back into the S columns as
+//               16-bit pairs (tcgen05.st). The running max m only moves when the row max passes
+//               it by more than 2^8, so every exponential stays <= 256; O and the row sum are
+//               then rescaled in TMEM (the commit that signalled S(u) also covers PV(u-1), so O
+//               is at rest). Epilogue: O / l, NaN for rows with no key, 0 past q_lengths.
+//
+// Every mbarrier wait is bounded (P.wait_timeout_ns); on a timeout the CTA records
+// SDPA_ERR_TIMEOUT in the status word, every role unwinds and the TMEM is released.
+#pragma once
+
+#include <cuda.h>
+
+#include <type_traits>
+
+#include "device_common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace sdpa {
+namespace prefill {
+
+using namespace sm100;
+
+constexpr int kBlockM = 128;
+constexpr int kBlockN = 128;
+constexpr int kThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer + MMA (+2 idle)
+// Register split (setmaxnreg): the two softmax warpgroups grow to kSoftmaxRegs, the last one
+// shrinks to kOtherRegs. 2*128*216 + 128*72 = 64512 = 384 * 168, the launch's registers; the
+// host refuses to launch unless the kernel was compiled with >= kLaunchRegs per thread.
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
+constexpr int kLaunchRegs = 168;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 bytes (64 16-bit columns)
+constexpr int kNone = 1 << 30;
+
+// bias / mask variants compiled into the kernel
+enum { kBiasNone = 0, kBiasSame = 1, kBiasF32 = 2 };
+enum { kMaskNone = 0, kMaskDense = 1, kMaskBits = 2 };
+
+template <int D>
+struct Cfg {
+  static constexpr int kRegions = D / 64;
+  static constexpr int kTileBytes = kRegions * kRegionBytes;
+  static constexpr int kKStages = D == 128 ? 2 : 4;
+  static constexpr int kVStages = D == 128 ? 2 : 4;
+  static constexpr int kBarriers = 2 * 2 + 2 * kKStages + 2 * kVStages + 2 * 4 + 1;
+  static constexpr int kSmemBytes = (2 + kKStages + kVStages) * kTileBytes + kBarriers * 8 + 64 + 1024;
+};
+
+struct TensorMaps {
+  CUtensorMap q, k, v;
+};
+
+// One query tile of a unit.
+struct QTile {
+  int h, qt, i0, n;      // n = number of key tiles it visits
+  const uint32_t* list;  // block list (kb | class << 30), or null for the prefix 0..n-1
+  __device__ __forceinline__ int kb(int j) const { return list ? (int)(list[j] & 0x3FFFFFFFu) : j; }
+  __device__ __forceinline__ int next(int j) const { return j < n ? kb(j) : kNone; }
+};
+
+struct Unit {
+  int b, kvh;
+  int q_len, kv_len, offset;
+  QTile t[2];
+};
+
+__device__ __forceinline__ QTile make_qtile(const Problem& P, const BatchInfo& bi, int h, int qt, bool present) {
+  QTile x;
+  x.h = h;
+  x.qt = qt;
+  x.i0 = qt * kBlockM;
+  x.list = nullptr;
+  x.n = 0;
+  if (!present || bi.skip || x.i0 >= bi.q_len) return x;
+  int n_lim = (bi.kv_len + kBlockN - 1) / kBlockN;
+  if (P.causal != SDPA_CAUSAL_NONE) {
+    const long long last_row = min(x.i0 + kBlockM - 1, bi.q_len - 1);
+    const long long last_key = (long long)bi.offset + last_row;
+    n_lim = last_key < 0 ? 0 : (int)min((long long)n_lim, last_key / kBlockN + 1);
+  }
+  if (P.bcls) {
+    const int hm = P.bi_nheads == 1 ? 0 : h;
+    const long long row = (long long)hm * P.bi_nqb + qt;
+    x.list = P.brow_list + row * P.bi_nkb;
+    const int cnt = P.brow_count[row];
+    int n = 0;
+    while (n < cnt && (int)(x.list[n] & 0x3FFFFFFFu) < n_lim) ++n;
+    x.n = n;
+  } else {
+    x.n = n_lim;
+  }
+  return x;
+}
+
+// Units: with GQA, (query tile, batch, kv head, head pair); without, (tile pair, batch, head).
+// Enumerated longest causal rows first.
+__host__ __device__ __forceinline__ int units_per_level(const Problem& P) {
+  return P.group >= 2 ? P.B * P.Hkv * ((P.group + 1) / 2) : P.B * P.H;
+}
+__host__ __device__ __forceinline__ int n_levels(const Problem& P) {
+  const int nqt = (P.Lq + kBlockM - 1) / kBlockM;
+  return P.group >= 2 ? nqt : (nqt + 1) / 2;
+}
+
+__device__ __forceinline__ Unit make_unit(const Problem& P, int u) {
+  Unit w;
+  const int per = units_per_level(P);
+  const int level = n_levels(P) - 1 - u / per;
+  const int rem = u % per;
+  const int nqt = (P.Lq + kBlockM - 1) / kBlockM;
+  int hA, hB, qA, qB;
+  bool haveB;
+  if (P.group >= 2) {
+    const int pairs = (P.group + 1) / 2;
+    w.b = rem / (P.Hkv * pairs);
+    const int r2 = rem % (P.Hkv * pairs);
+    w.kvh = r2 / pairs;
+    const int pr = r2 % pairs;
+    hA = w.kvh * P.group + 2 * pr;
+    hB = hA + 1;
+    haveB = 2 * pr + 1 < P.group;
+    qA = qB = level;
+  } else {
+    w.b = rem / P.H;
+    hA = hB = rem % P.H;
+    w.kvh = hA;
+    qA = 2 * level;
+    qB = qA + 1;
+    haveB = qB < nqt;
+  }
+  const BatchInfo bi = resolve_batch(P, w.b);
+  w.q_len = bi.q_len;
+  w.kv_len = bi.kv_len;
+  w.offset = bi.offset;
+  w.t[0] = make_qtile(P, bi, hA, qA, true);
+  w.t[1] = make_qtile(P, bi, hB, qB, haveB);
+  if (!haveB) w.t[1].i0 = kNone;  // marks "no tile B"
+  return w;
+}
+
+template <typename BT>
+__device__ __forceinline__ void load8(const BT* p, float (&f)[8]) {
+  if constexpr (std::is_same<BT, float>::value) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  } else {
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      BT lo, hi;
+      const uint16_t l16 = (uint16_t)(w[k] & 0xFFFFu), h16 = (uint16_t)(w[k] >> 16);
+      lo = *reinterpret_cast<const BT*>(&l16);
+      hi = *reinterpret_cast<const BT*>(&h16);
+      f[2 * k] = to_f32(lo);
+      f[2 * k + 1] = to_f32(hi);
+    }
+  }
+}
+
+template <typename T, int D, int kBias, int kMask>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __restrict__ out, int n_units) {
+  using C = Cfg<D>;
+  using BT = typename std::conditional<kBias == kBiasF32, float, T>::type;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_smem = smem;  // [2] tiles
+  uint8_t* k_smem = q_smem + 2 * C::kTileBytes;
+  uint8_t* v_smem = k_smem + C::kKStages * C::kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(v_smem + C::kVStages * C::kTileBytes);
+  uint64_t* q_full = bars;                  // [2]
+  uint64_t* q_empty = q_full + 2;           // [2]
+  uint64_t* k_full = q_empty + 2;           // [KS]
+  uint64_t* k_empty = k_full + C::kKStages;
+  uint64_t* v_full = k_empty + C::kKStages; // [VS]
+  uint64_t* v_empty = v_full + C::kVStages;
+  uint64_t* s_full = v_empty + C::kVStages; // [2]
+  uint64_t* p_full = s_full + 2;            // [2]
+  uint64_t* o_ready = p_full + 2;           // [2]
+  uint64_t* o_free = o_ready + 2;           // [2]
+  uint64_t* drain = o_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint64_t tmo = P.wait_timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], kBlockM);
+      mbar_init(&o_ready[s], 1);
+      mbar_init(&o_free[s], kBlockM);
+    }
+    for (int s = 0; s < C::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < C::kVStages; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.k);
+    prefetch_tmap(&maps.v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    report(P.status, SDPA_ERR_TIMEOUT);
+  };
+  // every lane of a warp takes the same branch; a timeout seen by any lane stops the warp
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const bool ok = mbar_wait(bar, parity, tmo, abort_flag);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    fail();
+    return false;
+  };
+  const bool elected = lane == 0;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
+  }
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    [&] {
+      uint32_t g = 0;            // key tiles loaded so far (ring position)
+      uint32_t qc[2] = {0, 0};   // Q tiles loaded per stream
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const Unit w = make_unit(P, u);
+        if (w.t[0].n == 0 && w.t[1].n == 0) continue;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (w.t[s].n == 0) continue;
+          if (!wait_all(&q_empty[s], (qc[s] & 1) ^ 1)) return;
+          if (elected) {
+            mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
+            for (int r = 0; r < C::kRegions; ++r)
+              tma_load_4d(q_smem + s * C::kTileBytes + r * kRegionBytes, &maps.q, &q_full[s], r * 64,
+                          w.t[s].h, w.t[s].i0, w.b);
+          }
+          ++qc[s];
+        }
+        // union of the two tiles' key lists; K_u is loaded ahead of V_{u-1}
+        int ja = 0, jb = 0, prev_kb = -1;
+        for (;;) {
+          const int na = w.t[0].next(ja), nb = w.t[1].next(jb);
+          const int kb = min(na, nb);
+          if (kb != kNone) {
+            const uint32_t x = g;
+            const int ks = x % C::kKStages;
+            if (!wait_all(&k_empty[ks], ((x / C::kKStages) & 1) ^ 1)) return;
+            if (elected) {
+              mbar_arrive_expect_tx(&k_full[ks], C::kTileBytes);
+              for (int r = 0; r < C::kRegions; ++r)
+                tma_load_4d(k_smem + ks * C::kTileBytes + r * kRegionBytes, &maps.k, &k_full[ks], r * 64,
+                            w.kvh, kb * kBlockN, w.b);
+            }
+          }
+          if (prev_kb >= 0) {
+            const uint32_t x = g - 1;
+            const int vs = x % C::kVStages;
+            if (!wait_all(&v_empty[vs], ((x / C::kVStages) & 1) ^ 1)) return;
+            if (elected) {
+              mbar_arrive_expect_tx(&v_full[vs], C::kTileBytes);
+              for (int r = 0; r < C::kRegions; ++r)
+                tma_load_4d(v_smem + vs * C::kTileBytes + r * kRegionBytes, &maps.v, &v_full[vs], r * 64,
+                            w.kvh, prev_kb * kBlockN, w.b);
+            }
+          }
+          __syncwarp();
+          if (kb == kNone) break;
+          if (na == kb) ++ja;
+          if (nb == kb) ++jb;
+          prev_kb = kb;
+          ++g;
+        }
+      }
+    }();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    [&] {
+      constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+      constexpr uint32_t idesc_qk = instr_desc_f16(kBf16, false, false, kBlockM, kBlockN);
+      constexpr uint32_t idesc_pv = instr_desc_f16(kBf16, false, true, kBlockM, D);
+      const uint32_t q_base = smem_addr(q_smem), k_base = smem_addr(k_smem), v_base = smem_addr(v_smem);
+      uint32_t g = 0;
+      uint32_t sc[2] = {0, 0};  // S tiles issued per stream (phase of s_full / p_full)
+      uint32_t qc[2] = {0, 0};
+      uint32_t oc[2] = {0, 0};  // units per stream (phase of o_ready / o_free)
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const Unit w = make_unit(P, u);
+        if (w.t[0].n == 0 && w.t[1].n == 0) continue;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (w.t[s].n == 0) continue;
+          if (!wait_all(&q_full[s], qc[s] & 1)) return;
+          ++qc[s];
+        }
+        bool pend[2] = {false, false};  // a PV of the previous key tile is owed
+        bool first_pv[2] = {true, true};
+        int ja = 0, jb = 0;
+        // PV of stream s for the key tile at ring position x (waits for its P)
+        auto pv = [&](int s, uint32_t x) -> bool {
+          if (!wait_all(&p_full[s], (sc[s] - 1) & 1)) return false;
+          const int vs = x % C::kVStages;
+          if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
+          if (first_pv[s] && !wait_all(&o_free[s], (oc[s] & 1) ^ 1)) return false;
+          tc_fence_after();
+          if (elected) {
+            const uint32_t vtile = v_base + vs * C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kBlockN / 16; ++kk) {
+              // B = V (keys x dims, dims contiguous): MN-major; 64-dim regions kRegionBytes
+              // apart (LBO), 8-key groups 1024 bytes apart (SBO); 16 keys per step.
+              const uint64_t bdesc = smem_desc_sw128(vtile + kk * 16 * 128, kRegionBytes, 1024);
+              mma_ts(tmem + 256 + s * D, tmem + s * 128 + kk * 8, bdesc, idesc_pv,
+                     (first_pv[s] && kk == 0) ? 0u : 1u);
+            }
+          }
+          __syncwarp();
+          first_pv[s] = false;
+          return true;
+        };
+        auto qk = [&](int s, int ks) {
+          tc_fence_after();
+          if (elected) {
+            const uint32_t qtile = q_base + s * C::kTileBytes, ktile = k_base + ks * C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              // A = Q, B = K: both K-major, 128-byte rows, 8-row groups 1024 bytes apart.
+              const uint32_t off = (kk / 4) * kRegionBytes + (kk % 4) * 32;
+              mma_ss(tmem + s * 128, smem_desc_sw128(qtile + off, 16, 1024),
+                     smem_desc_sw128(ktile + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&s_full[s]);
+          }
+          __syncwarp();
+          ++sc[s];
+        };
+        for (;;) {
+          const int na = w.t[0].next(ja), nb = w.t[1].next(jb);
+          const int kb = min(na, nb);
+          const bool in[2] = {kb != kNone && na == kb, kb != kNone && nb == kb};
+          const uint32_t x = g;  // ring position of this key tile
+          const int ks = x % C::kKStages;
+          if (kb != kNone && !wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
+  #pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (pend[s] && !pv(s, x - 1)) return;
+            if (in[s]) {
+              qk(s, ks);
+              // the stream's last S has been issued: Q_s may be reloaded once it completes
+              if (elected && (s == 0 ? ja : jb) + 1 == w.t[s].n) mma_commit(&q_empty[s]);
+            }
+          }
+          if (elected) {
+            if (pend[0] || pend[1]) mma_commit(&v_empty[(x - 1) % C::kVStages]);
+            if (kb != kNone) mma_commit(&k_empty[ks]);
+          }
+          __syncwarp();
+          if (kb == kNone) break;
+          pend[0] = in[0];
+          pend[1] = in[1];
+          if (in[0]) ++ja;
+          if (in[1]) ++jb;
+          ++g;
+        }
+        if (elected) {
+  #pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (w.t[s].n == 0) continue;
+            mma_commit(&o_ready[s]);
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          if (w.t[s].n != 0) ++oc[s];
+      }
+    }();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ softmax + epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
+    [&] {
+      const int s = warp / 4;            // stream (tile A or B)
+      const int r = threadIdx.x % 128;   // query row within the tile = TMEM lane
+      const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+      const uint32_t scol = s * 128, ocol = 256 + s * D;
+      const float sl2 = P.scale_log2;
+      uint32_t sc = 0, oc = 0;
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const Unit w = make_unit(P, u);
+        const QTile qt = s ? w.t[1] : w.t[0];
+        if (qt.i0 == kNone) continue;  // the unit has no tile B
+        const int i = qt.i0 + r;
+        T* orow = out + (((long long)w.b * P.Lq + i) * P.H + qt.h) * D;
+        if (qt.n == 0) {
+          // no key tile: NaN rows (nothing attended) or zero rows (past q_lengths)
+          if (i < P.Lq) {
+            const float val = (i >= w.q_len) ? 0.f : __int_as_float(0x7fc00000);
+            const uint32_t wv = std::is_same<T, __half>::value ? pack_f16x2(val, val) : pack_bf16x2(val, val);
+#pragma unroll
+            for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(wv, wv, wv, wv);
+          }
+          continue;
+        }
+        // keys j < row_lim are allowed by kv_lengths and the causal bound of this row; rows past
+        // q_lengths (or the array) attend nothing, so no bias / mask element is read for them
+        long long lim = (i < w.q_len) ? w.kv_len : 0;
+        if (P.causal != SDPA_CAUSAL_NONE) lim = min(lim, (long long)w.offset + i + 1);
+        const int row_lim = (int)max(lim, -1LL);
+        const BT* bias_row = nullptr;
+        if constexpr (kBias != kBiasNone)
+          bias_row = static_cast<const BT*>(P.bias) + (long long)i * P.bs[1] + (long long)qt.h * P.bs[2] +
+                     (long long)w.b * P.bs[3];
+        const uint8_t* mask_row = nullptr;
+        if constexpr (kMask == kMaskDense)
+          mask_row = P.mask + (long long)i * P.ms[1] + (long long)qt.h * P.ms[2] + (long long)w.b * P.ms[3];
+        float m_used = -INFINITY, l = 0.f;
+        for (int j = 0; j < qt.n; ++j) {
+          const int kb = qt.kb(j);
+          const int key0 = kb * kBlockN;
+          const int nvalid = min(max(row_lim - key0, 0), kBlockN);
+          uint32_t bw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+          if constexpr (kMask == kMaskBits) {
+            if ((qt.list[j] >> 30) == SDPA_BLOCK_PARTIAL && nvalid > 0) {
+              const int hm = P.bi_nheads == 1 ? 0 : qt.h;
+              const long long blk = ((long long)hm * P.bi_nqb + qt.qt) * P.bi_nkb + kb;
+              const uint4 b4 = *reinterpret_cast<const uint4*>(P.bbits + (blk * kBlockM + r) * 4);
+              bw[0] = b4.x; bw[1] = b4.y; bw[2] = b4.z; bw[3] = b4.w;
+            }
+          }
+          if (!wait_all(&s_full[s], sc & 1)) return;
+          ++sc;
+          tc_fence_after();
+          uint32_t v[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + scol + c * 32, v[c]);
+          tmem_wait_ld();
+          // logits in log2 units (masked: -inf) and the row max
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          const bool full_tile = (nvalid == kBlockN) && (kMask == kMaskNone ||
+                                 (kMask == kMaskBits && (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu));
+          if (kBias == kBiasNone && kMask != kMaskDense && full_tile) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const float t = __uint_as_float(v[c][e]) * sl2;
+                v[c][e] = __float_as_uint(t);
+                mx[e & 3] = fmaxf(mx[e & 3], t);
+              }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float bia[32];
+              uint32_t mk[8];
+              if constexpr (kBias != kBiasNone) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                  const int col = c * 32 + e;
+                  float f8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                  if (col + 8 <= nvalid) {
+                    load8<BT>(bias_row + key0 + col, f8);
+                  } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                      if (col + k < nvalid) f8[k] = to_f32(bias_row[key0 + col + k]);
+                  }
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) bia[e + k] = f8[k] * kLog2e;
+                }
+              }
+              if constexpr (kMask == kMaskDense) {
+                const int col = c * 32;
+                if (col + 32 <= nvalid) {
+                  const uint4 a = *reinterpret_cast<const uint4*>(mask_row + key0 + col);
+                  const uint4 b = *reinterpret_cast<const uint4*>(mask_row + key0 + col + 16);
+                  mk[0] = a.x; mk[1] = a.y; mk[2] = a.z; mk[3] = a.w; mk[4] = b.x; mk[5] = b.y; mk[6] = b.z; mk[7] = b.w;
+                } else {
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) {
+                    uint32_t wd = 0;
+#pragma unroll
+                    for (int y = 0; y < 4; ++y)
+                      if (col + 4 * k + y < nvalid) wd |= (uint32_t)(mask_row[key0 + col + 4 * k + y] != 0) << (8 * y);
+                    mk[k] = wd;
+                  }
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int col = c * 32 + e;
+                float t = __uint_as_float(v[c][e]) * sl2;
+                if constexpr (kBias != kBiasNone) t += bia[e];
+                bool ok = col < nvalid;
+                if constexpr (kMask == kMaskBits) ok = ok && ((bw[c] >> e) & 1u);
+                if constexpr (kMask == kMaskDense) ok = ok && ((mk[e / 4] >> (8 * (e % 4))) & 0xFFu);
+                t = ok ? t : -INFINITY;
+                v[c][e] = __float_as_uint(t);
+                mx[e & 3] = fmaxf(mx[e & 3], t);
+              }
+            }
+          }
+          const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+          // the running max moves only when the row max passes it by 2^8 (or leaves -inf)
+          const bool grow = (rmax > m_used + kRescaleThreshold) || (m_used == -INFINITY && rmax != -INFINITY);
+          float alpha = 1.f;
+          if (grow) {
+            alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - rmax);
+            m_used = rmax;
+          }
+          const bool need_o = grow && alpha != 0.f && j > 0;
+          if (__any_sync(0xffffffffu, need_o)) {
+            // O holds PV of the earlier key tiles (complete: the S commit covered them)
+            const float a = need_o ? alpha : 1.f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(lane_addr + ocol + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
+              tmem_st32(lane_addr + ocol + c * 32, o);
+            }
+            tmem_wait_st();
+          }
+          l *= alpha;
+          const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+          // P = 2^(t - m), 16-bit pairs into the first 64 columns of the tile's S columns
+          float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float p0 = ex2(__uint_as_float(v[c][e]) - msub);
+              const float p1 = ex2(__uint_as_float(v[c][e + 1]) - msub);
+              rs[(e >> 1) & 3] += p0 + p1;
+              pk[e / 2] = std::is_same<T, __half>::value ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[c / 2][(c % 2) * 16 + e] = pk[e];
+          }
+          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+          tmem_st32(lane_addr + scol, v[0]);
+          tmem_st32(lane_addr + scol + 32, v[1]);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_full[s]);
+        }
+        if (!wait_all(&o_ready[s], oc & 1)) return;
+        ++oc;
+        tc_fence_after();
+        const bool pad = i >= w.q_len;
+        const float inv = (l > 0.f) ? 1.f / l : __int_as_float(0x7fc00000);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + ocol + c * 32, o);
+          tmem_wait_ld();
+          if (i < P.Lq) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t wv[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k]) * inv : inv);
+                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k + 1]) * inv : inv);
+                wv[k] = std::is_same<T, __half>::value ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
+              }
+              *reinterpret_cast<uint4*>(orow + c * 32 + e) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&o_free[s]);
+      }
+    }();
+  }
+  if (warp == 9) {
+    // every MMA this CTA issued has completed before its TMEM is released (also on a timeout)
+    if (elected) mma_commit(drain);
+    __syncwarp();
+    mbar_wait(drain, 0, tmo, nullptr);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Host launcher for one (T, D) pair; defined in the per-type translation units.
+template <typename T, int D>
+cudaError_t launch(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream);
+template <> cudaError_t launch<__nv_bfloat16, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch<__half, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch<__half, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+
+template <typename T, int D, int kBias, int kMask>
+cudaError_t launch_variant(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream) {
+  auto kern = prefill_kernel<T, D, kBias, kMask>;
+  const int smem = Cfg<D>::kSmemBytes;
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  // setmaxnreg.inc would wait forever if the launch held fewer registers than the split needs
+  if (attr.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int n_units = units_per_level(P) * n_levels(P);
+  kern<<<grid, kThreads, smem, stream>>>(maps, P, static_cast<T*>(out), n_units);
+  return cudaGetLastError();
+}
+
+inline int bias_variant(const Problem& P) {
+  if (!P.bias) return kBiasNone;
+  return P.bias_dtype == SDPA_F32 ? kBiasF32 : kBiasSame;
+}
+inline int mask_variant(const Problem& P) {
+  if (P.bcls) return kMaskBits;
+  if (P.mask) return kMaskDense;
+  return kMaskNone;
+}
+
+#define SDPA_PREFILL_DEFINE_LAUNCH(T, D)                                                              \
+  template <>                                                                                       \
+  cudaError_t launch<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,         \
+                           cudaStream_t stream) {                                                   \
+    const int b = bias_variant(P), m = mask_variant(P);                                             \
+    switch (b * 3 + m) {                                                                            \
+      case 0: return launch_variant<T, D, kBiasNone, kMaskNone>(maps, P, out, grid, stream);        \
+      case 1: return launch_variant<T, D, kBiasNone, kMaskDense>(maps, P, out, grid, stream);       \
+      case 2: return launch_variant<T, D, kBiasNone, kMaskBits>(maps, P, out, grid, stream);        \
+      case 3: return launch_variant<T, D, kBiasSame, kMaskNone>(maps, P, out, grid, stream);        \
+      case 4: return launch_variant<T, D, kBiasSame, kMaskDense>(maps, P, out, grid, stream);       \
+      case 5: return launch_variant<T, D, kBiasSame, kMaskBits>(maps, P, out, grid, stream);        \
+      case 6: return launch_variant<T, D, kBiasF32, kMaskNone>(maps, P, out, grid, stream);         \
+      case 7: return launch_variant<T, D, kBiasF32, kMaskDense>(maps, P, out, grid, stream);        \
+      default: return launch_variant<T, D, kBiasF32, kMaskBits>(maps, P, out, grid, stream);       \
+    }                                                                                               \
+  }
+
+}  // namespace prefill
+}  // namespace sdpa

@@ -95,6 +95,7 @@ sdpa_status resolve(const sdpa_params* p, sdpa::Problem* P) {
     P->ms[d] = p->mask_stride[d];
   }
   P->mask = p->mask;
+  P->wait_timeout_ns = 1000000000ull;  // 1 s: far beyond any legitimate wait
   if (bi) {
     P->bcls = bi->block_class;
     P->brow_count = bi->row_count;

@@ -55,7 +55,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 255u) == 0) {
-      if (*abort) return false;
+      if (abort && *abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) return false;
     }
   }
