@@ -98,9 +98,13 @@ def test_prefill_block_info():
     out = run(q, k, v, block_info=info)
     want = oracle.sdpa_forward(f64(q), f64(k), f64(v), mask=mask.cpu().numpy()[None])
     assert_matches(out, want, 1e-2, "block info")
-    # the dense-mask path of the same kernel agrees
-    out2 = run(q, k, v, mask=mask)
+    # the dense mask itself (900 keys per row: not 16-byte aligned, so the SIMT kernel) agrees
+    out2 = sdpa.sdpa_forward(q.to(DEV), k.to(DEV), v.to(DEV), mask=mask)
     assert_matches(out2, want, 1e-2, "dense mask")
+    # an aligned dense mask goes through the tcgen05 kernel's dense-mask variant
+    out3 = run(q[:, :, :, :], k[:, :896], v[:, :896], mask=mask[:, :, :896].contiguous())
+    want3 = oracle.sdpa_forward(f64(q), f64(k[:, :896]), f64(v[:, :896]), mask=mask[:, :, :896].cpu().numpy()[None])
+    assert_matches(out3, want3, 1e-2, "dense mask (tcgen05)")
 
 
 def test_prefill_empty_rows_and_all_masked_blocks():
