@@ -48,6 +48,9 @@ struct BatchInfo {
   bool skip;   // decode: the cache index is out of range, leave this sequence alone
 };
 
+// Records the message sdpa_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 // Launchers (each returns a cudaError_t from the launch).
 cudaError_t launch_generic(const Problem& P, const void* q, const void* k, const void* v,
                            void* out, cudaStream_t stream);

@@ -124,6 +124,10 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+namespace sdpa {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace sdpa
+
 extern "C" {
 
 size_t sdpa_workspace_size(const sdpa_params* p) {

@@ -164,6 +164,29 @@ SDPA_API sdpa_status sdpa_decode_with_cache(const sdpa_params* p, const void* q,
                                    const int32_t* cache_index, void* out, void* ws,
                                    size_t ws_bytes, struct CUstream_st* stream);
 
+/* Decoding with a KV cache for callers that cannot allocate device memory (this entry point
+ * has no counterpart in the paper). Some callers cannot call cudaMalloc: plug-ins hosted by a
+ * framework that owns every device allocation, or latency-critical decode loops that must never
+ * block on, or fail in, the allocator mid-run. They cannot supply the workspace that
+ * sdpa_decode_with_cache needs. This call computes the same thing, with the same arguments
+ * minus the workspace. Its scratch is a fixed array of SDPA_STATIC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads the library holds until the process exits.
+ *  - A call whose scratch need (sdpa_workspace_size(p)) exceeds that size is rejected with
+ *    SDPA_ERR_WORKSPACE before anything is launched.
+ *  - The first call on each device looks up the array's device address with that device
+ *    current. Make that first call before any stream capture.
+ *  - Every call on a device shares the one array. Calls that overlap on the GPU (other streams,
+ *    other host threads) race on it: serialise them.
+ *  - The device status word sits in the array and is cleared at the start of each call. The
+ *    caller cannot read it. An out-of-range cache_index still skips that sequence.
+ *  - Nothing is allocated. No cudaMalloc, cudaFree or allocating library routine is called. */
+#define SDPA_STATIC_SCRATCH_BYTES (32u << 20)
+SDPA_API sdpa_status sdpa_decode_with_cache_static(const sdpa_params* p, const void* q,
+                                                   const void* k_new, const void* v_new,
+                                                   void* k_cache, void* v_cache,
+                                                   const int32_t* cache_index, void* out,
+                                                   struct CUstream_st* stream);
+
 /* Writes k_new/v_new [batch][n_new][nkvheads][d] of `dtype` into the caches
  * [batch][capacity][nkvheads][d] at rows index[b] + t, t < n_new (index: device
  * int32[batch]). Either cache pair may be NULL to update only the other. An index outside
