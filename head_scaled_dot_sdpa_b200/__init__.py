@@ -37,6 +37,7 @@ STATUS_NAMES = {0: "SDPA_OK", 1: "SDPA_ERR_INVALID_ARG", 2: "SDPA_ERR_UNSUPPORTE
 SDPA_F32, SDPA_F16, SDPA_BF16 = 0, 1, 2
 SDPA_CAUSAL_NONE, SDPA_CAUSAL_TOP_LEFT, SDPA_CAUSAL_BOTTOM_RIGHT = 0, 1, 2
 SDPA_FLAG_GENERIC_KERNEL = 0x1
+SDPA_FLAG_SELFTEST_STALL = 0x2
 SDPA_BLOCK_EMPTY, SDPA_BLOCK_PARTIAL, SDPA_BLOCK_FULL = 0, 1, 2
 
 _DTYPE = {torch.float32: SDPA_F32, torch.float16: SDPA_F16, torch.bfloat16: SDPA_BF16}
@@ -239,14 +240,15 @@ def _check_qkv(q, k, v):
 
 def sdpa_forward(q, k, v, bias=None, *, mask=None, scale=None, is_causal=False, q_offset=0,
                  q_lengths=None, kv_lengths=None, block_info=None, out=None, workspace=None,
-                 generic=False, stream=None):
+                 generic=False, flags=0, stream=None):
     """scaled_dot_product_attention(q, k, v, [bias]; mask, scale, is_causal, q_offset,
-    q_lengths, kv_lengths) — is_causal is False, True or "bottom_right"."""
+    q_lengths, kv_lengths) — is_causal is False, True or "bottom_right". `flags` takes extra
+    SDPA_FLAG_* bits (e.g. the bounded-wait self-test)."""
     _check_qkv(q, k, v)
     keep = []
     p = _params(q, k, v, bias=bias, mask=mask, scale=scale, is_causal=is_causal, q_offset=q_offset,
                 q_lengths=q_lengths, kv_lengths=kv_lengths, block_info=block_info,
-                flags=SDPA_FLAG_GENERIC_KERNEL if generic else 0, keep=keep)
+                flags=(SDPA_FLAG_GENERIC_KERNEL if generic else 0) | flags, keep=keep)
     if out is None:
         out = torch.empty(q.shape[:3] + (v.shape[3],), dtype=q.dtype, device=q.device)
     need = _lib.sdpa_workspace_size(ctypes.byref(p))

@@ -38,6 +38,7 @@ struct Problem {
   int bi_nheads, bi_nqb, bi_nkb, bi_bq, bi_bk;
   int* status;               // device status word (never null when a kernel runs)
   unsigned long long wait_timeout_ns;  // bound on every mbarrier wait of the tcgen05 kernel
+  int selftest_stall;                  // SDPA_FLAG_SELFTEST_STALL
 };
 
 // Per-batch values every kernel resolves the same way.

@@ -58,6 +58,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 bytes (64 16-bit columns)
 constexpr int kNone = 1 << 30;
+constexpr int kUnitSlots = 4;        // ring of unit indices handed from the producer to the others
+constexpr int kUnitConsumers = 9;    // the MMA warp and the 8 softmax warps
+constexpr int kSchedWord = 16;       // int offset in the status area of the unit counter (+1: done)
 
 // bias / mask variants compiled into the kernel
 enum { kBiasNone = 0, kBiasSame = 1, kBiasF32 = 2 };
@@ -69,7 +72,7 @@ struct Cfg {
   static constexpr int kTileBytes = kRegions * kRegionBytes;
   static constexpr int kKStages = D == 128 ? 2 : 4;
   static constexpr int kVStages = D == 128 ? 2 : 4;
-  static constexpr int kBarriers = 2 * 2 + 2 * kKStages + 2 * kVStages + 2 * 4 + 1;
+  static constexpr int kBarriers = 2 * 2 + 2 * kKStages + 2 * kVStages + 2 * 4 + 1 + 2 * kUnitSlots;
   static constexpr int kSmemBytes = (2 + kKStages + kVStages) * kTileBytes + kBarriers * 8 + 64 + 1024;
 };
 
@@ -208,7 +211,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint64_t* o_ready = p_full + 2;           // [2]
   uint64_t* o_free = o_ready + 2;           // [2]
   uint64_t* drain = o_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* unit_full = drain + 1;               // [kUnitSlots]
+  uint64_t* unit_empty = unit_full + kUnitSlots; // [kUnitSlots]
+  int* unit_ring = reinterpret_cast<int*>(unit_empty + kUnitSlots);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring + kUnitSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -226,6 +232,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     for (int s = 0; s < C::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < C::kVStages; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
     mbar_init(drain, 1);
+    for (int k = 0; k < kUnitSlots; ++k) {
+      mbar_init(&unit_full[k], 1);
+      mbar_init(&unit_empty[k], kUnitConsumers);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -255,6 +265,17 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     return false;
   };
   const bool elected = lane == 0;
+  // Dynamic scheduling: the producer takes units from a counter in the workspace (units are
+  // numbered longest causal rows first) and hands them to the other roles through a small ring.
+  unsigned int* sched = reinterpret_cast<unsigned int*>(P.status) + kSchedWord;
+  auto next_unit = [&](uint32_t k, int& u) -> bool {  // consumers: the k-th unit of this CTA
+    const int slot = k % kUnitSlots;
+    if (!wait_all(&unit_full[slot], (k / kUnitSlots) & 1)) return false;
+    u = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+    __syncwarp();
+    if (elected) mbar_arrive(&unit_empty[slot]);
+    return true;
+  };
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
@@ -264,7 +285,20 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     [&] {
       uint32_t g = 0;            // key tiles loaded so far (ring position)
       uint32_t qc[2] = {0, 0};   // Q tiles loaded per stream
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      // self-test: wait for a phase no one completes (the consumers' first release of slot 0)
+      if (P.selftest_stall && !wait_all(&unit_empty[0], 0)) return;
+      for (uint32_t k = 0;; ++k) {
+        const int slot = k % kUnitSlots;
+        if (!wait_all(&unit_empty[slot], ((k / kUnitSlots) & 1) ^ 1)) return;
+        int u = 0;
+        if (elected) {
+          u = (int)atomicAdd(sched, 1u);
+          if (u > n_units) u = n_units;
+          unit_ring[slot] = u;
+          mbar_arrive(&unit_full[slot]);
+        }
+        u = __shfl_sync(0xffffffffu, u, 0);
+        if (u >= n_units) break;
         const Unit w = make_unit(P, u);
         if (w.t[0].n == 0 && w.t[1].n == 0) continue;
 #pragma unroll
@@ -326,7 +360,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       uint32_t sc[2] = {0, 0};  // S tiles issued per stream (phase of s_full / p_full)
       uint32_t qc[2] = {0, 0};
       uint32_t oc[2] = {0, 0};  // units per stream (phase of o_ready / o_free)
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      for (uint32_t kq = 0;; ++kq) {
+        int u;
+        if (!next_unit(kq, u)) return;
+        if (u >= n_units) break;
         const Unit w = make_unit(P, u);
         if (w.t[0].n == 0 && w.t[1].n == 0) continue;
 #pragma unroll
@@ -427,7 +464,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
       uint32_t sc = 0, oc = 0;
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      for (uint32_t kq = 0;; ++kq) {
+        int u;
+        if (!next_unit(kq, u)) return;
+        if (u >= n_units) break;
         const Unit w = make_unit(P, u);
         const QTile qt = s ? w.t[1] : w.t[0];
         if (qt.i0 == kNone) continue;  // the unit has no tile B
@@ -476,20 +516,23 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + scol + c * 32, v[c]);
           tmem_wait_ld();
-          // logits in log2 units (masked: -inf) and the row max
+          // Fast path (no bias, no mask bytes, every key of the tile attended by every row of
+          // the warp): v keeps the raw scores, the max is taken on them (scale > 0) and the
+          // exponent argument is one packed FMA, s * scale*log2e - m. Otherwise v becomes the
+          // logits in log2 units, -inf where masked, and the argument is v - m.
           float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          const bool full_tile = (nvalid == kBlockN) && (kMask == kMaskNone ||
-                                 (kMask == kMaskBits && (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu));
-          if (kBias == kBiasNone && kMask != kMaskDense && full_tile) {
+          const bool full_row = (nvalid == kBlockN) && (kMask == kMaskNone ||
+                                (kMask == kMaskBits && (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu));
+          const bool fast = kBias == kBiasNone && kMask != kMaskDense && __all_sync(0xffffffffu, full_row);
+          float mul;
+          if (fast) {
+            mul = sl2;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const float t = __uint_as_float(v[c][e]) * sl2;
-                v[c][e] = __float_as_uint(t);
-                mx[e & 3] = fmaxf(mx[e & 3], t);
-              }
+              for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[c][e]));
           } else {
+            mul = 1.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               float bia[32];
@@ -541,7 +584,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               }
             }
           }
-          const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+          const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * mul;
           // the running max moves only when the row max passes it by 2^8 (or leaves -inf)
           const bool grow = (rmax > m_used + kRescaleThreshold) || (m_used == -INFINITY && rmax != -INFINITY);
           float alpha = 1.f;
@@ -565,17 +608,24 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             tmem_wait_st();
           }
           l *= alpha;
-          const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-          // P = 2^(t - m), 16-bit pairs into the first 64 columns of the tile's S columns
+          const float negm = (m_used == -INFINITY) ? 0.f : -m_used;
+          // P = 2^(v * mul - m), 16-bit pairs into the first 64 columns of the tile's S columns.
+          // On the fast path every fourth pair is computed on the FMA pipe instead of the MUFU.
           float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2(__uint_as_float(v[c][e]) - msub);
-              const float p1 = ex2(__uint_as_float(v[c][e + 1]) - msub);
-              rs[(e >> 1) & 3] += p0 + p1;
+              float x0, x1, p0, p1;
+              fma2(x0, x1, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), mul, mul, negm, negm);
+              if (((e >> 1) & 3) == 3 && fast) {
+                exp2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              add2(rs[(e >> 1) & 2], rs[((e >> 1) & 2) + 1], rs[(e >> 1) & 2], rs[((e >> 1) & 2) + 1], p0, p1);
               pk[e / 2] = std::is_same<T, __half>::value ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
             }
 #pragma unroll
@@ -629,6 +679,15 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  // the last CTA to finish resets the unit counter for the next launch on this workspace
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(sched, 0u);
+      atomicExch(sched + 1, 0u);
+      __threadfence();
+    }
   }
 }
 

@@ -96,6 +96,10 @@ sdpa_status resolve(const sdpa_params* p, sdpa::Problem* P) {
   }
   P->mask = p->mask;
   P->wait_timeout_ns = 1000000000ull;  // 1 s: far beyond any legitimate wait
+  if (p->flags & SDPA_FLAG_SELFTEST_STALL) {
+    P->wait_timeout_ns = 1000000ull;  // 1 ms
+    P->selftest_stall = 1;
+  }
   if (bi) {
     P->bcls = bi->block_class;
     P->brow_count = bi->row_count;

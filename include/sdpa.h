@@ -91,6 +91,10 @@ typedef struct sdpa_block_mask_info {
 
 /* Flags (sdpa_params.flags). */
 #define SDPA_FLAG_GENERIC_KERNEL 0x1u /* force the SIMT kernel (any dtype / head size) */
+/* Self-test of the bounded waits (tests only): every mbarrier wait of the tcgen05 kernel is
+ * limited to 1 ms and its TMA producer first waits on a barrier that nothing completes, so the
+ * call ends early with SDPA_ERR_TIMEOUT in the status word and the context stays usable. */
+#define SDPA_FLAG_SELFTEST_STALL 0x2u
 
 /* One attention call. Arguments of the page's entry and where they sit here:
  *  dtype            element type of q, k, v and out (fp32 accumulation throughout; out is

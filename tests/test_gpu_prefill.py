@@ -131,3 +131,17 @@ def test_unaligned_mask_takes_the_simt_kernel():
     assert sdpa.last_kernel() == "generic_simt"
     want = oracle.sdpa_forward(f64(q), f64(k), f64(v), mask=mask.numpy())
     assert_matches(out, want, 1e-2, "unaligned mask")
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """Every mbarrier wait of the tcgen05 kernel is bounded. The self-test flag makes the TMA
+    producer wait on a phase nothing completes (with 1 ms bounds): the call must end with
+    SDPA_ERR_TIMEOUT in the status word, and the next call must run normally."""
+    q, k, v = _qkv(12, 1, 256, 256, 2, 2, 128, torch.bfloat16)
+    ws = sdpa.Workspace(DEV)
+    sdpa.sdpa_forward(q.to(DEV), k.to(DEV), v.to(DEV), workspace=ws, flags=sdpa.SDPA_FLAG_SELFTEST_STALL)
+    assert sdpa.last_kernel() == "prefill_tcgen05"
+    assert sdpa.read_device_status(ws) == sdpa.SDPA_ERR_TIMEOUT
+    out = sdpa.sdpa_forward(q.to(DEV), k.to(DEV), v.to(DEV), workspace=ws)
+    assert sdpa.read_device_status(ws) == sdpa.SDPA_OK
+    assert_matches(out, oracle.sdpa_forward(f64(q), f64(k), f64(v)), 1e-2, "after the timeout")
