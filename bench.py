@@ -53,6 +53,36 @@ def causal_pairs(Lq, Lk, offset=0):
     return int(np.clip(offset + i + 1, 0, Lk).sum())
 
 
+# ---- ncu figures committed under profiles/ ------------------------------------------------------
+
+PREFILL_SOURCES = ("prefill_sm100.cuh", "sm100_primitives.cuh", "prefill_sm100.cu")
+
+
+def source_hash(names):
+    """sha256 (first 16 hex digits) of the kernel's source files, in the given order."""
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "head_scaled_dot_sdpa_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(summary, sources):
+    """DRAM bytes per launch recorded in a profiles/ summary, or None when the summary is
+    missing or was taken on other kernel sources than the current ones."""
+    import re
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    mh = re.search(r"source hash:\s*`?([0-9a-f]{16})", text)
+    mt = re.search(r"dram bytes per launch:\s*`?([0-9]+)", text)
+    if not mh or not mt or mh.group(1) != source_hash(sources):
+        return None
+    return int(mt.group(1))
+
+
 # ---- distributed plumbing -------------------------------------------------------------------
 
 def init_dist(n_gpus):
@@ -206,11 +236,7 @@ def run_ours(args, rank, world, local):
     h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
     d2h = out.numel() * out.element_size()
 
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            traffic = json.load(f).get("prefill_tcgen05", None)
+    traffic = profiled_traffic("prefill_tcgen05_causal_gqa_prefill.md", PREFILL_SOURCES)
 
     result.update({
         "metric": "prefill attention TFLOP/s (unmasked FLOPs)",
@@ -255,8 +281,23 @@ def other_workloads(args, dev, world, ws, peaks):
     import head_scaled_dot_sdpa_b200 as sdpa
 
     res = {}
-    # KV-cache decode: HBM GB/s over the bytes a step must move
+    if "decode" in args.workloads:
+        res["kv_cache_decode"] = decode_workload(args, dev, world, ws, peaks)
+    if "bias" in args.workloads:
+        res["alibi_t5_bias"] = bias_workload(args, dev, world, ws)
+    if "block_sparse" in args.workloads:
+        res["block_sparse_mask"] = block_sparse_workload(args, dev, world, ws, peaks)
+    return res
+
+
+def decode_workload(args, dev, world, ws, peaks):
+    """KV-cache decode: HBM GB/s over the bytes a step must move."""
+    import dataclasses
+    import head_scaled_dot_sdpa_b200 as sdpa
+
     w = si.KV_CACHE_DECODE
+    if args.shrink > 1:
+        w = dataclasses.replace(w, batch=max(1, w.batch // args.shrink))
     d = si.decode_inputs(w)
     qd, kn, vn = d["q"].to(dev), d["k_new"].to(dev), d["v_new"].to(dev)
     kc, vc = d["k_cache"].to(dev), d["v_cache"].to(dev)
@@ -268,14 +309,17 @@ def other_workloads(args, dev, world, ws, peaks):
     per = time_steps(step, args.steps, args.warmup, world)
     ms = max_over_ranks(float(np.mean(per)), world)
     gbs = byts / (ms * 1e-3) / 1e9
-    res["kv_cache_decode"] = {"workload": w.name, "metric": "decode HBM GB/s", "value": round(gbs * world, 1),
-                              "unit": "GB/s", "ms_per_step": round(ms, 4), "bytes_per_step": byts,
-                              "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"],
-                                           "unit": "GB/s", "frac": round(gbs / peaks["hbm"], 4)},
-                              "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 4}
-    del qd, kn, vn, kc, vc, out
+    return {"workload": w.name, "metric": "decode HBM GB/s", "value": round(gbs * world, 1),
+            "unit": "GB/s", "ms_per_step": round(ms, 4), "bytes_per_step": byts, "batch": w.batch,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm"], 4)},
+            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 4}
 
-    # ALiBi/T5 bias attention
+
+def bias_workload(args, dev, world, ws):
+    """ALiBi/T5 bias attention (fp16, causal, additive bias)."""
+    import head_scaled_dot_sdpa_b200 as sdpa
+
     w = si.ALIBI_T5_BIAS
     q, k, v = [t.to(dev) for t in si.qkv(w)]
     bias = si.alibi_t5_bias(w).to(dev)
@@ -285,13 +329,19 @@ def other_workloads(args, dev, world, ws, peaks):
     per = time_steps(step, args.steps, args.warmup, world)
     ms = max_over_ranks(float(np.mean(per)), world)
     bias_bytes = w.nheads * causal_pairs(w.q_len, w.kv_len) * 2
-    res["alibi_t5_bias"] = {"workload": w.name, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2),
-                            "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
-                            "bias_GBs": round(bias_bytes / (ms * 1e-3) / 1e9, 1), "kernel": sdpa.last_kernel()}
-    del q, k, v, bias, out
+    return {"workload": w.name, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2),
+            "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "bias_GBs": round(bias_bytes / (ms * 1e-3) / 1e9, 1), "kernel": sdpa.last_kernel()}
 
-    # block-sparse mask: classification pass + attention over the non-empty blocks
+
+def block_sparse_workload(args, dev, world, ws, peaks):
+    """Block-sparse mask: the classification pass, then attention over the non-empty blocks."""
+    import dataclasses
+    import head_scaled_dot_sdpa_b200 as sdpa
+
     w = si.BLOCK_SPARSE
+    if args.shrink > 1:
+        w = dataclasses.replace(w, q_len=w.q_len // args.shrink, kv_len=w.kv_len // args.shrink)
     cls = si.block_classes(w)
     mask = si.mask_device(w, cls, dev)
     allowed = int(mask.sum(dtype=torch.int64).item())
@@ -306,13 +356,12 @@ def other_workloads(args, dev, world, ws, peaks):
     ms = max_over_ranks(float(np.mean(per)), world)
     flops = 4.0 * w.head_dim * allowed
     n_blocks = int((cls != 0).sum())
-    res["block_sparse_mask"] = {
-        "workload": w.name, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2), "unit": "TFLOP/s (unmasked)",
+    return {
+        "workload": w.name, "q_len": w.q_len, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2), "unit": "TFLOP/s (unmasked)",
         "ms_per_step": round(ms, 4), "executed_tflops": round(4.0 * w.head_dim * n_blocks * 128 * 128 / (ms * 1e-3) / 1e12, 2),
         "classification": {"ms": round(ms_c, 4), "GB/s": round(mask.numel() / (ms_c * 1e-3) / 1e9, 1),
                            "frac_hbm": round(mask.numel() / (ms_c * 1e-3) / 1e9 / peaks["hbm"], 4)},
         "kernel": sdpa.last_kernel()}
-    return res
 
 
 # ---- CPU oracle ---------------------------------------------------------------------------------
@@ -395,6 +444,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--reference-heads", type=int, default=16)
+    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse",
+                    help="comma list; without 'prefill' only the other workloads run (a profiling aid)")
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="divide the decode batch and the block-sparse length by this (small ncu cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -407,9 +460,16 @@ def main():
         print(json.dumps(run_reference(args, rank, world)), flush=True)
         return
 
+    args.workloads = set(x.strip() for x in args.workloads.split(",") if x.strip())
     rank, world, local = init_dist(args.gpus)
     try:
-        res = run_ours(args, rank, world, local)
+        if "prefill" in args.workloads:
+            res = run_ours(args, rank, world, local)
+        else:
+            torch.cuda.set_device(local)
+            import head_scaled_dot_sdpa_b200 as sdpa
+            res = {"other_workloads": other_workloads(args, torch.device("cuda", local), world,
+                                                      sdpa.Workspace(torch.device("cuda", local)), _peaks())}
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
