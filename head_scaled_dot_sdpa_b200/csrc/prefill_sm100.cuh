@@ -3,33 +3,29 @@
 // section "Fused implementation": tile by tile, online softmax over key tiles, weights never
 // materialised), for fp16/bf16 inputs with qk_head_dim = v_head_dim in {64, 128}.
 //
-// Work unit: one 128-query tile of one (batch, query head). Persistent CTAs (one per SM) take
-// units from a counter, longest causal rows first, the query heads of one key/value group next
-// to each other (their K/V tiles then come from L2). A unit visits its key tiles in order: the
-// causal / kv_lengths prefix, or the non-empty blocks of a block-sparse mask.
-//
-// TMEM (512 columns): two S slots of 128 fp32 columns, P (64 columns of 16-bit pairs), O.
-// Because S is double-buffered and P has its own columns, the tensor core computes
-// S(u+1) = Q K(u+1)^T while the softmax works on S(u); the time per key tile is the larger of
-// the softmax time and the MMA time instead of their sum.
+// Work unit: two 128-query tiles A and B that read the same key/value head of the same batch
+// element: two query heads of one GQA group (same query tile), or, without GQA, two adjacent
+// query tiles of one head. Persistent CTAs (one per SM) walk the units, longest causal rows
+// first. The key tiles a unit visits are the union of the two tiles' lists (the causal /
+// kv_lengths prefix, or the non-empty blocks of a block-sparse mask), each loaded once.
 //
 // Warp roles (384 threads):
-//   warp 8      TMA producer: Q (double-buffered across units), K(u) ahead of V(u-1), through
-//               128B-swizzled rings; it also takes units from the counter and hands them out;
+//   warp 8      TMA producer: Q_A, Q_B, then K_u ahead of V_{u-1} through 128B-swizzled rings;
 //   warp 9      MMA issuer and TMEM owner (warps 10-11 idle; warpgroup 2 gives its registers to
 //               the softmax warpgroups with setmaxnreg). Per key tile u, in this order:
-//                 S(u) = Q K(u)^T into slot u%2      (both operands in shared memory)
-//                 O += P(u-1) V(u-1)                  (P read from TMEM)
-//   warps 0-7   softmax: each query row (= TMEM lane) is split between two threads, warpgroup h
-//               taking keys [64h, 64h+64) of the tile and output columns [hD/2, hD/2 + D/2):
-//               tcgen05.ld of its half row (the S slot is released right after); masks
-//               (causal / q_offset / kv_lengths as one prefix bound per row, boolean mask bytes
-//               or partial-block bits); optional bias; the half's max, combined with the other
-//               half through shared memory; P = 2^(s*scale*log2e - m) stored as 16-bit pairs
-//               (tcgen05.st) once the previous PV has read P. The running max m only moves when
-//               the row max passes it by more than 2^8, so every exponential stays <= 256; O
-//               and the row sum are then rescaled in TMEM (after the previous PV completed).
-//               Epilogue: O / l, NaN for rows with no key, 0 past q_lengths.
+//                 O_A += P_A(u-1) V(u-1);  S_A(u) = Q_A K(u)^T;
+//                 O_B += P_B(u-1) V(u-1);  S_B(u) = Q_B K(u)^T
+//               (S: tcgen05.mma with both operands in shared memory; PV: P read from TMEM). So
+//               the tensor pipe works on one tile while the other tile's softmax runs, and the
+//               in-order tcgen05 pipeline lets S_X(u) reuse the columns PV_X(u-1) just read;
+//   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: one thread per query row
+//               (= TMEM lane). tcgen05.ld of the S row; masks (causal / q_offset / kv_lengths
+//               as one prefix bound per row, boolean mask bytes or partial-block bits); optional
+//               bias; row max; P = 2^(s*scale*log2e - m) written back into the S columns as
+//               16-bit pairs (tcgen05.st). The running max m only moves when the row max passes
+//               it by more than 2^8, so every exponential stays <= 256; O and the row sum are
+//               then rescaled in TMEM (the commit that signalled S(u) also covers PV(u-1), so O
+//               is at rest). Epilogue: O / l, NaN for rows with no key, 0 past q_lengths.
 //
 // Every mbarrier wait is bounded (P.wait_timeout_ns); on a timeout the CTA records
 // SDPA_ERR_TIMEOUT in the status word, every role unwinds and the TMEM is released.
@@ -50,26 +46,22 @@ using namespace sm100;
 
 constexpr int kBlockM = 128;
 constexpr int kBlockN = 128;
-constexpr int kThreads = 384;  // 3 warpgroups: softmax half 0, softmax half 1, producer + MMA (+2 idle)
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer + MMA (+2 idle)
 // Register split (setmaxnreg): the two softmax warpgroups grow to kSoftmaxRegs, the last one
-// shrinks to kOtherRegs. 2*128*184 + 128*136 = 64512 = 384 * 168, the launch's registers; the
+// shrinks to kOtherRegs. 2*128*216 + 128*72 = 64512 = 384 * 168, the launch's registers; the
 // host refuses to launch unless the kernel was compiled with >= kLaunchRegs per thread.
-constexpr int kSoftmaxRegs = 184;
-constexpr int kOtherRegs = 136;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
 constexpr int kLaunchRegs = 168;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kPCol = 256;  // P: 64 columns
-constexpr uint32_t kOCol = 320;  // O: D columns
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 bytes (64 16-bit columns)
-constexpr int kUnitSlots = 4;              // ring of unit indices handed from the producer
-constexpr int kUnitConsumers = 9;          // the MMA warp and the 8 softmax warps
-constexpr int kSchedWord = 16;             // int offset in the status area of the unit counter (+1: done)
-constexpr int kSoftmaxThreads = 256;
+constexpr int kNone = 1 << 30;
+constexpr int kUnitSlots = 4;        // ring of unit indices handed from the producer to the others
+constexpr int kUnitConsumers = 9;    // the MMA warp and the 8 softmax warps
+constexpr int kSchedWord = 16;       // int offset in the status area of the unit counter (+1: done)
 
 // bias / mask variants compiled into the kernel
 enum { kBiasNone = 0, kBiasSame = 1, kBiasF32 = 2 };
@@ -79,67 +71,101 @@ template <int D>
 struct Cfg {
   static constexpr int kRegions = D / 64;
   static constexpr int kTileBytes = kRegions * kRegionBytes;
-  static constexpr int kQStages = 2;
   static constexpr int kKStages = D == 128 ? 2 : 4;
   static constexpr int kVStages = D == 128 ? 2 : 4;
-  // q full/empty, k, v, s full/free, p_full, pv_done, o_ready, o_free, max/sum exchange, drain,
-  // unit ring
-  static constexpr int kBarriers = 2 * kQStages + 2 * kKStages + 2 * kVStages + 2 * 2 + 4 + 3 + 1 + 2 * kUnitSlots;
-  // tiles, barriers, unit ring + TMEM address + abort flag, the max / sum exchange buffers
-  // (3 x 2 x kBlockM floats), and slack to align the base to 1024 bytes
-  static constexpr int kSmemBytes = (kQStages + kKStages + kVStages) * kTileBytes + kBarriers * 8 + 64 +
-                                    6 * kBlockM * 4 + 1024;
+  static constexpr int kBarriers = 2 * 2 + 2 * kKStages + 2 * kVStages + 2 * 4 + 1 + 2 * kUnitSlots;
+  static constexpr int kSmemBytes = (2 + kKStages + kVStages) * kTileBytes + kBarriers * 8 + 64 + 1024;
 };
 
 struct TensorMaps {
   CUtensorMap q, k, v;
 };
 
-// One unit: a 128-query tile of (batch b, query head h).
-struct Unit {
-  int b, h, kvh, qt, i0, n;  // n = number of key tiles it visits
-  int q_len, kv_len, offset;
-  const uint32_t* list;      // block list (kb | class << 30), or null for the prefix 0..n-1
+// One query tile of a unit.
+struct QTile {
+  int h, qt, i0, n;      // n = number of key tiles it visits
+  const uint32_t* list;  // block list (kb | class << 30), or null for the prefix 0..n-1
   __device__ __forceinline__ int kb(int j) const { return list ? (int)(list[j] & 0x3FFFFFFFu) : j; }
+  __device__ __forceinline__ int next(int j) const { return j < n ? kb(j) : kNone; }
 };
 
-// Units are numbered (query tile descending, batch, kv head, head within the group).
-__host__ __device__ __forceinline__ int units_per_level(const Problem& P) { return P.B * P.H; }
-__host__ __device__ __forceinline__ int n_levels(const Problem& P) { return (P.Lq + kBlockM - 1) / kBlockM; }
+struct Unit {
+  int b, kvh;
+  int q_len, kv_len, offset;
+  QTile t[2];
+};
 
-__device__ __forceinline__ Unit make_unit(const Problem& P, int u) {
-  Unit w;
-  const int per = units_per_level(P);
-  w.qt = n_levels(P) - 1 - u / per;
-  const int rem = u % per;
-  w.b = rem / P.H;
-  w.h = rem % P.H;  // heads of one group are consecutive: h / group = kv head
-  w.kvh = w.h / P.group;
-  w.i0 = w.qt * kBlockM;
-  const BatchInfo bi = resolve_batch(P, w.b);
-  w.q_len = bi.q_len;
-  w.kv_len = bi.kv_len;
-  w.offset = bi.offset;
-  w.list = nullptr;
-  w.n = 0;
-  if (bi.skip || w.i0 >= bi.q_len) return w;
+__device__ __forceinline__ QTile make_qtile(const Problem& P, const BatchInfo& bi, int h, int qt, bool present) {
+  QTile x;
+  x.h = h;
+  x.qt = qt;
+  x.i0 = qt * kBlockM;
+  x.list = nullptr;
+  x.n = 0;
+  if (!present || bi.skip || x.i0 >= bi.q_len) return x;
   int n_lim = (bi.kv_len + kBlockN - 1) / kBlockN;
   if (P.causal != SDPA_CAUSAL_NONE) {
-    const long long last_row = min(w.i0 + kBlockM - 1, bi.q_len - 1);
+    const long long last_row = min(x.i0 + kBlockM - 1, bi.q_len - 1);
     const long long last_key = (long long)bi.offset + last_row;
     n_lim = last_key < 0 ? 0 : (int)min((long long)n_lim, last_key / kBlockN + 1);
   }
   if (P.bcls) {
-    const int hm = P.bi_nheads == 1 ? 0 : w.h;
-    const long long row = (long long)hm * P.bi_nqb + w.qt;
-    w.list = P.brow_list + row * P.bi_nkb;
+    const int hm = P.bi_nheads == 1 ? 0 : h;
+    const long long row = (long long)hm * P.bi_nqb + qt;
+    x.list = P.brow_list + row * P.bi_nkb;
     const int cnt = P.brow_count[row];
     int n = 0;
-    while (n < cnt && (int)(w.list[n] & 0x3FFFFFFFu) < n_lim) ++n;
-    w.n = n;
+    while (n < cnt && (int)(x.list[n] & 0x3FFFFFFFu) < n_lim) ++n;
+    x.n = n;
   } else {
-    w.n = n_lim;
+    x.n = n_lim;
   }
+  return x;
+}
+
+// Units: with GQA, (query tile, batch, kv head, head pair); without, (tile pair, batch, head).
+// Enumerated longest causal rows first.
+__host__ __device__ __forceinline__ int units_per_level(const Problem& P) {
+  return P.group >= 2 ? P.B * P.Hkv * ((P.group + 1) / 2) : P.B * P.H;
+}
+__host__ __device__ __forceinline__ int n_levels(const Problem& P) {
+  const int nqt = (P.Lq + kBlockM - 1) / kBlockM;
+  return P.group >= 2 ? nqt : (nqt + 1) / 2;
+}
+
+__device__ __forceinline__ Unit make_unit(const Problem& P, int u) {
+  Unit w;
+  const int per = units_per_level(P);
+  const int level = n_levels(P) - 1 - u / per;
+  const int rem = u % per;
+  const int nqt = (P.Lq + kBlockM - 1) / kBlockM;
+  int hA, hB, qA, qB;
+  bool haveB;
+  if (P.group >= 2) {
+    const int pairs = (P.group + 1) / 2;
+    w.b = rem / (P.Hkv * pairs);
+    const int r2 = rem % (P.Hkv * pairs);
+    w.kvh = r2 / pairs;
+    const int pr = r2 % pairs;
+    hA = w.kvh * P.group + 2 * pr;
+    hB = hA + 1;
+    haveB = 2 * pr + 1 < P.group;
+    qA = qB = level;
+  } else {
+    w.b = rem / P.H;
+    hA = hB = rem % P.H;
+    w.kvh = hA;
+    qA = 2 * level;
+    qB = qA + 1;
+    haveB = qB < nqt;
+  }
+  const BatchInfo bi = resolve_batch(P, w.b);
+  w.q_len = bi.q_len;
+  w.kv_len = bi.kv_len;
+  w.offset = bi.offset;
+  w.t[0] = make_qtile(P, bi, hA, qA, true);
+  w.t[1] = make_qtile(P, bi, hB, qB, haveB);
+  if (!haveB) w.t[1].i0 = kNone;  // marks "no tile B"
   return w;
 }
 
@@ -154,9 +180,12 @@ __device__ __forceinline__ void load8(const BT* p, float (&f)[8]) {
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
+      BT lo, hi;
       const uint16_t l16 = (uint16_t)(w[k] & 0xFFFFu), h16 = (uint16_t)(w[k] >> 16);
-      f[2 * k] = to_f32(*reinterpret_cast<const BT*>(&l16));
-      f[2 * k + 1] = to_f32(*reinterpret_cast<const BT*>(&h16));
+      lo = *reinterpret_cast<const BT*>(&l16);
+      hi = *reinterpret_cast<const BT*>(&h16);
+      f[2 * k] = to_f32(lo);
+      f[2 * k + 1] = to_f32(hi);
     }
   }
 }
@@ -168,48 +197,41 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   using BT = typename std::conditional<kBias == kBiasF32, float, T>::type;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_smem = smem;
-  uint8_t* k_smem = q_smem + C::kQStages * C::kTileBytes;
+  uint8_t* q_smem = smem;  // [2] tiles
+  uint8_t* k_smem = q_smem + 2 * C::kTileBytes;
   uint8_t* v_smem = k_smem + C::kKStages * C::kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(v_smem + C::kVStages * C::kTileBytes);
-  uint64_t* q_full = bars;                         // [QS]
-  uint64_t* q_empty = q_full + C::kQStages;        // [QS]
-  uint64_t* k_full = q_empty + C::kQStages;        // [KS]
+  uint64_t* q_full = bars;                  // [2]
+  uint64_t* q_empty = q_full + 2;           // [2]
+  uint64_t* k_full = q_empty + 2;           // [KS]
   uint64_t* k_empty = k_full + C::kKStages;
-  uint64_t* v_full = k_empty + C::kKStages;        // [VS]
+  uint64_t* v_full = k_empty + C::kKStages; // [VS]
   uint64_t* v_empty = v_full + C::kVStages;
-  uint64_t* s_full = v_empty + C::kVStages;        // [2] S slot computed
-  uint64_t* s_free = s_full + 2;                   // [2] S slot read by the softmax
-  uint64_t* p_full = s_free + 2;                   // P written
-  uint64_t* pv_done = p_full + 1;                  // PV completed (P free, O at rest)
-  uint64_t* o_ready = pv_done + 1;
-  uint64_t* o_free = o_ready + 1;
-  uint64_t* xmax = o_free + 1;                     // [2] half-row maxima exchanged (by parity)
-  uint64_t* xsum = xmax + 2;                       // half-row sums exchanged
-  uint64_t* drain = xsum + 1;
-  uint64_t* unit_full = drain + 1;                 // [kUnitSlots]
-  uint64_t* unit_empty = unit_full + kUnitSlots;   // [kUnitSlots]
+  uint64_t* s_full = v_empty + C::kVStages; // [2]
+  uint64_t* p_full = s_full + 2;            // [2]
+  uint64_t* o_ready = p_full + 2;           // [2]
+  uint64_t* o_free = o_ready + 2;           // [2]
+  uint64_t* drain = o_free + 2;
+  uint64_t* unit_full = drain + 1;               // [kUnitSlots]
+  uint64_t* unit_empty = unit_full + kUnitSlots; // [kUnitSlots]
   int* unit_ring = reinterpret_cast<int*>(unit_empty + kUnitSlots);
-  float* red_max = reinterpret_cast<float*>(unit_ring + kUnitSlots);  // [parity][half][row]
-  float* red_sum = red_max + 2 * 2 * kBlockM;                         // [half][row]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_sum + 2 * kBlockM);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring + kUnitSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint64_t tmo = P.wait_timeout_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kQStages; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], kBlockM);
+      mbar_init(&o_ready[s], 1);
+      mbar_init(&o_free[s], kBlockM);
+    }
     for (int s = 0; s < C::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < C::kVStages; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_free[s], kSoftmaxThreads); }
-    mbar_init(p_full, kSoftmaxThreads);
-    mbar_init(pv_done, 1);
-    mbar_init(o_ready, 1);
-    mbar_init(o_free, kSoftmaxThreads);
-    mbar_init(&xmax[0], kSoftmaxThreads);
-    mbar_init(&xmax[1], kSoftmaxThreads);
-    mbar_init(xsum, kSoftmaxThreads);
     mbar_init(drain, 1);
     for (int k = 0; k < kUnitSlots; ++k) {
       mbar_init(&unit_full[k], 1);
@@ -218,11 +240,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tmap(&maps.q);
     prefetch_tmap(&maps.k);
     prefetch_tmap(&maps.v);
@@ -244,8 +266,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     return false;
   };
   const bool elected = lane == 0;
-  // Dynamic scheduling: the producer takes units from a counter in the workspace and hands
-  // them to the other roles through a small ring.
+  // Dynamic scheduling: the producer takes units from a counter in the workspace (units are
+  // numbered longest causal rows first) and hands them to the other roles through a small ring.
   unsigned int* sched = reinterpret_cast<unsigned int*>(P.status) + kSchedWord;
   auto next_unit = [&](uint32_t k, int& u) -> bool {  // consumers: the k-th unit of this CTA
     const int slot = k % kUnitSlots;
@@ -256,13 +278,14 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     return true;
   };
 
-  if (warp >= kProducerWarp) {
+  if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
   }
-  if (warp == kProducerWarp) {
+  if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     [&] {
-      uint32_t g = 0, qc = 0;  // key tiles and Q tiles loaded so far
+      uint32_t g = 0;            // key tiles loaded so far (ring position)
+      uint32_t qc[2] = {0, 0};   // Q tiles loaded per stream
       // self-test: wait for a phase no one completes (the consumers' first release of slot 0)
       if (P.selftest_stall && !wait_all(&unit_empty[0], 0)) return;
       for (uint32_t k = 0;; ++k) {
@@ -278,141 +301,186 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         u = __shfl_sync(0xffffffffu, u, 0);
         if (u >= n_units) break;
         const Unit w = make_unit(P, u);
-        if (w.n == 0) continue;
-        const int qs = qc % C::kQStages;
-        if (!wait_all(&q_empty[qs], ((qc / C::kQStages) & 1) ^ 1)) return;
-        if (elected) {
-          mbar_arrive_expect_tx(&q_full[qs], C::kTileBytes);
-          for (int r = 0; r < C::kRegions; ++r)
-            tma_load_4d(q_smem + qs * C::kTileBytes + r * kRegionBytes, &maps.q, &q_full[qs], r * 64, w.h,
-                        w.i0, w.b);
+        if (w.t[0].n == 0 && w.t[1].n == 0) continue;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (w.t[s].n == 0) continue;
+          if (!wait_all(&q_empty[s], (qc[s] & 1) ^ 1)) return;
+          if (elected) {
+            mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
+            for (int r = 0; r < C::kRegions; ++r)
+              tma_load_4d(q_smem + s * C::kTileBytes + r * kRegionBytes, &maps.q, &q_full[s], r * 64,
+                          w.t[s].h, w.t[s].i0, w.b);
+          }
+          ++qc[s];
         }
-        ++qc;
-        // K(j) is loaded ahead of V(j-1): the MMA needs S(j) before PV(j-1)
-        for (int j = 0; j <= w.n; ++j) {
-          if (j < w.n) {
-            const uint32_t x = g + j;
+        // union of the two tiles' key lists; K_u is loaded ahead of V_{u-1}
+        int ja = 0, jb = 0, prev_kb = -1;
+        for (;;) {
+          const int na = w.t[0].next(ja), nb = w.t[1].next(jb);
+          const int kb = min(na, nb);
+          if (kb != kNone) {
+            const uint32_t x = g;
             const int ks = x % C::kKStages;
             if (!wait_all(&k_empty[ks], ((x / C::kKStages) & 1) ^ 1)) return;
             if (elected) {
               mbar_arrive_expect_tx(&k_full[ks], C::kTileBytes);
               for (int r = 0; r < C::kRegions; ++r)
-                tma_load_4d(k_smem + ks * C::kTileBytes + r * kRegionBytes, &maps.k, &k_full[ks], r * 64, w.kvh,
-                            w.kb(j) * kBlockN, w.b);
+                tma_load_4d(k_smem + ks * C::kTileBytes + r * kRegionBytes, &maps.k, &k_full[ks], r * 64,
+                            w.kvh, kb * kBlockN, w.b);
             }
           }
-          if (j >= 1) {
-            const uint32_t x = g + j - 1;
+          if (prev_kb >= 0) {
+            const uint32_t x = g - 1;
             const int vs = x % C::kVStages;
             if (!wait_all(&v_empty[vs], ((x / C::kVStages) & 1) ^ 1)) return;
             if (elected) {
               mbar_arrive_expect_tx(&v_full[vs], C::kTileBytes);
               for (int r = 0; r < C::kRegions; ++r)
-                tma_load_4d(v_smem + vs * C::kTileBytes + r * kRegionBytes, &maps.v, &v_full[vs], r * 64, w.kvh,
-                            w.kb(j - 1) * kBlockN, w.b);
+                tma_load_4d(v_smem + vs * C::kTileBytes + r * kRegionBytes, &maps.v, &v_full[vs], r * 64,
+                            w.kvh, prev_kb * kBlockN, w.b);
             }
           }
           __syncwarp();
+          if (kb == kNone) break;
+          if (na == kb) ++ja;
+          if (nb == kb) ++jb;
+          prev_kb = kb;
+          ++g;
         }
-        g += w.n;
       }
     }();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     [&] {
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_qk = instr_desc_f16(kBf16, false, false, kBlockM, kBlockN);
       constexpr uint32_t idesc_pv = instr_desc_f16(kBf16, false, true, kBlockM, D);
       const uint32_t q_base = smem_addr(q_smem), k_base = smem_addr(k_smem), v_base = smem_addr(v_smem);
-      uint32_t g = 0, qc = 0, oc = 0;
-      // O += P(x) V(x); `first`: the unit's first PV (O is overwritten once the epilogue freed it)
-      auto pv = [&](uint32_t x, bool first) -> bool {
-        if (!wait_all(p_full, x & 1)) return false;
-        const int vs = x % C::kVStages;
-        if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
-        if (first && !wait_all(o_free, (oc & 1) ^ 1)) return false;
-        tc_fence_after();
-        if (elected) {
-          const uint32_t vtile = v_base + vs * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk) {
-            // B = V (keys x dims, dims contiguous): MN-major; 64-dim regions kRegionBytes
-            // apart (LBO), 8-key groups 1024 bytes apart (SBO); 16 keys per step.
-            const uint64_t bdesc = smem_desc_sw128(vtile + kk * 16 * 128, kRegionBytes, 1024);
-            mma_ts(tmem + kOCol, tmem + kPCol + kk * 8, bdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
-          }
-          mma_commit(pv_done);
-          mma_commit(&v_empty[vs]);
-        }
-        __syncwarp();
-        return true;
-      };
+      uint32_t g = 0;
+      uint32_t sc[2] = {0, 0};  // S tiles issued per stream (phase of s_full / p_full)
+      uint32_t qc[2] = {0, 0};
+      uint32_t oc[2] = {0, 0};  // units per stream (phase of o_ready / o_free)
       for (uint32_t kq = 0;; ++kq) {
         int u;
         if (!next_unit(kq, u)) return;
         if (u >= n_units) break;
         const Unit w = make_unit(P, u);
-        if (w.n == 0) continue;
-        const int qs = qc % C::kQStages;
-        if (!wait_all(&q_full[qs], (qc / C::kQStages) & 1)) return;
-        const uint32_t qtile = q_base + qs * C::kTileBytes;
-        for (int j = 0; j < w.n; ++j) {
-          const uint32_t x = g + j;
-          const int slot = x & 1;
-          const int ks = x % C::kKStages;
-          if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
-          // the softmax has read the slot's previous S
-          if (x >= 2 && !wait_all(&s_free[slot], ((x >> 1) - 1) & 1)) return;
+        if (w.t[0].n == 0 && w.t[1].n == 0) continue;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (w.t[s].n == 0) continue;
+          if (!wait_all(&q_full[s], qc[s] & 1)) return;
+          ++qc[s];
+        }
+        bool pend[2] = {false, false};  // a PV of the previous key tile is owed
+        bool first_pv[2] = {true, true};
+        int ja = 0, jb = 0;
+        // PV of stream s for the key tile at ring position x (waits for its P)
+        auto pv = [&](int s, uint32_t x) -> bool {
+          if (!wait_all(&p_full[s], (sc[s] - 1) & 1)) return false;
+          const int vs = x % C::kVStages;
+          if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
+          if (first_pv[s] && !wait_all(&o_free[s], (oc[s] & 1) ^ 1)) return false;
           tc_fence_after();
           if (elected) {
-            const uint32_t ktile = k_base + ks * C::kTileBytes;
+            const uint32_t vtile = v_base + vs * C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kBlockN / 16; ++kk) {
+              // B = V (keys x dims, dims contiguous): MN-major; 64-dim regions kRegionBytes
+              // apart (LBO), 8-key groups 1024 bytes apart (SBO); 16 keys per step.
+              const uint64_t bdesc = smem_desc_sw128(vtile + kk * 16 * 128, kRegionBytes, 1024);
+              mma_ts(tmem + 256 + s * D, tmem + s * 128 + kk * 8, bdesc, idesc_pv,
+                     (first_pv[s] && kk == 0) ? 0u : 1u);
+            }
+          }
+          __syncwarp();
+          first_pv[s] = false;
+          return true;
+        };
+        auto qk = [&](int s, int ks) {
+          tc_fence_after();
+          if (elected) {
+            const uint32_t qtile = q_base + s * C::kTileBytes, ktile = k_base + ks * C::kTileBytes;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               // A = Q, B = K: both K-major, 128-byte rows, 8-row groups 1024 bytes apart.
               const uint32_t off = (kk / 4) * kRegionBytes + (kk % 4) * 32;
-              mma_ss(tmem + slot * 128, smem_desc_sw128(qtile + off, 16, 1024),
+              mma_ss(tmem + s * 128, smem_desc_sw128(qtile + off, 16, 1024),
                      smem_desc_sw128(ktile + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
             }
-            mma_commit(&s_full[slot]);
-            mma_commit(&k_empty[ks]);
-            if (j + 1 == w.n) mma_commit(&q_empty[qs]);  // Q may be reloaded once S completes
+            mma_commit(&s_full[s]);
           }
           __syncwarp();
-          if (j >= 1 && !pv(x - 1, j == 1)) return;
+          ++sc[s];
+        };
+        for (;;) {
+          const int na = w.t[0].next(ja), nb = w.t[1].next(jb);
+          const int kb = min(na, nb);
+          const bool in[2] = {kb != kNone && na == kb, kb != kNone && nb == kb};
+          const uint32_t x = g;  // ring position of this key tile
+          const int ks = x % C::kKStages;
+          if (kb != kNone && !wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
+  #pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (pend[s] && !pv(s, x - 1)) return;
+            if (in[s]) {
+              qk(s, ks);
+              // the stream's last S has been issued: Q_s may be reloaded once it completes
+              if (elected && (s == 0 ? ja : jb) + 1 == w.t[s].n) mma_commit(&q_empty[s]);
+            }
+          }
+          if (elected) {
+            if (pend[0] || pend[1]) mma_commit(&v_empty[(x - 1) % C::kVStages]);
+            if (kb != kNone) mma_commit(&k_empty[ks]);
+          }
+          __syncwarp();
+          if (kb == kNone) break;
+          pend[0] = in[0];
+          pend[1] = in[1];
+          if (in[0]) ++ja;
+          if (in[1]) ++jb;
+          ++g;
         }
-        if (!pv(g + w.n - 1, w.n == 1)) return;
-        if (elected) mma_commit(o_ready);
+        if (elected) {
+  #pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (w.t[s].n == 0) continue;
+            mma_commit(&o_ready[s]);
+          }
+        }
         __syncwarp();
-        g += w.n;
-        ++qc;
-        ++oc;
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          if (w.t[s].n != 0) ++oc[s];
       }
     }();
-  } else if (warp < kProducerWarp) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax + epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
     [&] {
-      const int hf = warp / 4;                  // key / output-column half
-      const int r = (warp % 4) * 32 + lane;     // query row within the tile = TMEM lane
+      const int s = warp / 4;            // stream (tile A or B)
+      const int r = threadIdx.x % 128;   // query row within the tile = TMEM lane
       const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
-      const uint32_t pcol = kPCol + hf * 32;
-      const uint32_t ocol = kOCol + hf * (D / 2);
+      const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
-      uint32_t x = 0, oc = 0;  // key tiles seen, units finished
+      uint32_t sc = 0, oc = 0;
       for (uint32_t kq = 0;; ++kq) {
         int u;
         if (!next_unit(kq, u)) return;
         if (u >= n_units) break;
         const Unit w = make_unit(P, u);
-        const int i = w.i0 + r;
-        T* orow = out + (((long long)w.b * P.Lq + i) * P.H + w.h) * D + hf * (D / 2);
-        if (w.n == 0) {
+        const QTile qt = s ? w.t[1] : w.t[0];
+        if (qt.i0 == kNone) continue;  // the unit has no tile B
+        const int i = qt.i0 + r;
+        T* orow = out + (((long long)w.b * P.Lq + i) * P.H + qt.h) * D;
+        if (qt.n == 0) {
           // no key tile: NaN rows (nothing attended) or zero rows (past q_lengths)
           if (i < P.Lq) {
             const float val = (i >= w.q_len) ? 0.f : __int_as_float(0x7fc00000);
             const uint32_t wv = std::is_same<T, __half>::value ? pack_f16x2(val, val) : pack_bf16x2(val, val);
 #pragma unroll
-            for (int c = 0; c < D / 2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(wv, wv, wv, wv);
+            for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(wv, wv, wv, wv);
           }
           continue;
         }
@@ -423,57 +491,52 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         const int row_lim = (int)max(lim, -1LL);
         const BT* bias_row = nullptr;
         if constexpr (kBias != kBiasNone)
-          bias_row = static_cast<const BT*>(P.bias) + (long long)i * P.bs[1] + (long long)w.h * P.bs[2] +
+          bias_row = static_cast<const BT*>(P.bias) + (long long)i * P.bs[1] + (long long)qt.h * P.bs[2] +
                      (long long)w.b * P.bs[3];
         const uint8_t* mask_row = nullptr;
         if constexpr (kMask == kMaskDense)
-          mask_row = P.mask + (long long)i * P.ms[1] + (long long)w.h * P.ms[2] + (long long)w.b * P.ms[3];
+          mask_row = P.mask + (long long)i * P.ms[1] + (long long)qt.h * P.ms[2] + (long long)w.b * P.ms[3];
         float m_used = -INFINITY, l = 0.f;
-        for (int j = 0; j < w.n; ++j, ++x) {
-          const int kb = w.kb(j);
-          const int key0 = kb * kBlockN + hf * 64;  // first key of this thread's half
-          const int nvalid = min(max(row_lim - key0, 0), 64);
-          uint32_t bw[2] = {0xffffffffu, 0xffffffffu};
+        for (int j = 0; j < qt.n; ++j) {
+          const int kb = qt.kb(j);
+          const int key0 = kb * kBlockN;
+          const int nvalid = min(max(row_lim - key0, 0), kBlockN);
+          uint32_t bw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
           if constexpr (kMask == kMaskBits) {
-            if ((w.list[j] >> 30) == SDPA_BLOCK_PARTIAL && nvalid > 0) {
-              const int hm = P.bi_nheads == 1 ? 0 : w.h;
-              const long long blk = ((long long)hm * P.bi_nqb + w.qt) * P.bi_nkb + kb;
-              const uint2 b2 = *reinterpret_cast<const uint2*>(P.bbits + (blk * kBlockM + r) * 4 + hf * 2);
-              bw[0] = b2.x;
-              bw[1] = b2.y;
+            if ((qt.list[j] >> 30) == SDPA_BLOCK_PARTIAL && nvalid > 0) {
+              const int hm = P.bi_nheads == 1 ? 0 : qt.h;
+              const long long blk = ((long long)hm * P.bi_nqb + qt.qt) * P.bi_nkb + kb;
+              const uint4 b4 = *reinterpret_cast<const uint4*>(P.bbits + (blk * kBlockM + r) * 4);
+              bw[0] = b4.x; bw[1] = b4.y; bw[2] = b4.z; bw[3] = b4.w;
             }
           }
-          const int slot = x & 1;
-          if (!wait_all(&s_full[slot], (x >> 1) & 1)) return;
+          if (!wait_all(&s_full[s], sc & 1)) return;
+          ++sc;
           tc_fence_after();
-          uint32_t v[2][32];
-          tmem_ld32(lane_addr + slot * 128 + hf * 64, v[0]);
-          tmem_ld32(lane_addr + slot * 128 + hf * 64 + 32, v[1]);
+          uint32_t v[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + scol + c * 32, v[c]);
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(&s_free[slot]);  // the slot may take S(x+2)
-          // Fast path (no bias, no mask bytes, all 64 keys attended by every row of the warp):
-          // the max is taken on the raw scores (scale > 0) and the exponent argument is one
-          // packed FMA, s * scale*log2e - m. Otherwise v becomes the logits in log2 units, -inf
-          // where masked, and the argument is v - m.
-          float mx[2] = {-INFINITY, -INFINITY};
-          const bool full_row = (nvalid == 64) && (kMask == kMaskNone ||
-                                (kMask == kMaskBits && (bw[0] & bw[1]) == 0xffffffffu));
+          // Fast path (no bias, no mask bytes, every key of the tile attended by every row of
+          // the warp): v keeps the raw scores, the max is taken on them (scale > 0) and the
+          // exponent argument is one packed FMA, s * scale*log2e - m. Otherwise v becomes the
+          // logits in log2 units, -inf where masked, and the argument is v - m.
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          const bool full_row = (nvalid == kBlockN) && (kMask == kMaskNone ||
+                                (kMask == kMaskBits && (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu));
           const bool fast = kBias == kBiasNone && kMask != kMaskDense && __all_sync(0xffffffffu, full_row);
           float mul;
           if (fast) {
             mul = sl2;
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-              for (int e = 0; e < 32; e += 4) {
-                mx[0] = fmax3(mx[0], __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
-                mx[1] = fmax3(mx[1], __uint_as_float(v[c][e + 2]), __uint_as_float(v[c][e + 3]));
-              }
+              for (int e = 0; e < 32; e += 2)
+                mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
           } else {
             mul = 1.f;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 4; ++c) {
               float bia[32];
               uint32_t mk[8];
               if constexpr (kBias != kBiasNone) {
@@ -519,22 +582,15 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                 if constexpr (kMask == kMaskDense) ok = ok && ((mk[e / 4] >> (8 * (e % 4))) & 0xFFu);
                 t = ok ? t : -INFINITY;
                 v[c][e] = __float_as_uint(t);
-                mx[e & 1] = fmaxf(mx[e & 1], t);
+                mx[e & 3] = fmaxf(mx[e & 3], t);
               }
             }
           }
-          // combine the two halves' maxima through shared memory (double-buffered by tile
-          // parity, so one barrier per tile suffices)
-          // (an mbarrier rather than a barrier instruction: the wait is bounded)
-          const int par = x & 1;
-          red_max[(par * 2 + hf) * kBlockM + r] = fmaxf(mx[0], mx[1]) * mul;
-          mbar_arrive(&xmax[par]);
-          if (!wait_all(&xmax[par], (x >> 1) & 1)) return;
-          const float rmax = fmaxf(red_max[(par * 2 + hf) * kBlockM + r], red_max[(par * 2 + (hf ^ 1)) * kBlockM + r]);
-          // The running max moves only when the row max passes it by 2^8 (or leaves -inf); O
-          // (this thread's columns) and l are then rescaled, once the previous PV has completed.
-          // alpha may underflow to 0 when the max jumps by more than 2^126: O is then cleared.
+          const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * mul;
+          // the running max moves only when the row max passes it by 2^8 (or leaves -inf)
           const bool grow = (rmax > m_used + kRescaleThreshold) || (m_used == -INFINITY && rmax != -INFINITY);
+          // O needs rescaling when it holds terms taken against a finite max (alpha may
+          // underflow to 0 when the max jumps by more than 2^126: O is then cleared)
           const bool had_max = m_used != -INFINITY;
           float alpha = 1.f;
           if (grow) {
@@ -542,14 +598,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             m_used = rmax;
           }
           const bool need_o = grow && had_max && j > 0;
-          bool pv_waited = false;
           if (__any_sync(0xffffffffu, need_o)) {
-            if (!wait_all(pv_done, (x - 1) & 1)) return;  // PV(x-1): O at rest
-            pv_waited = true;
-            tc_fence_after();
+            // O holds PV of the earlier key tiles (complete: the S commit covered them)
             const float a = need_o ? alpha : 1.f;
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
               tmem_ld32(lane_addr + ocol + c * 32, o);
               tmem_wait_ld();
@@ -561,40 +614,36 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
           l *= alpha;
           const float negm = (m_used == -INFINITY) ? 0.f : -m_used;
-          // P = 2^(v * mul - m) as 16-bit pairs, packed in place (pair e of chunk c lands in
-          // v[0][c*16 + e/2], already consumed)
+          // P = 2^(v * mul - m), 16-bit pairs into the first 64 columns of the tile's S columns.
           float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
               float x0, x1;
               fma2(x0, x1, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), mul, mul, negm, negm);
               const float p0 = ex2(x0), p1 = ex2(x1);
               add2(rs[(e >> 1) & 2], rs[((e >> 1) & 2) + 1], rs[(e >> 1) & 2], rs[((e >> 1) & 2) + 1], p0, p1);
-              v[0][c * 16 + e / 2] = std::is_same<T, __half>::value ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+              pk[e / 2] = std::is_same<T, __half>::value ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
             }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[c / 2][(c % 2) * 16 + e] = pk[e];
+          }
           l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-          // P's columns are free once PV(x-1) has read them
-          if (x > 0 && !pv_waited && !wait_all(pv_done, (x - 1) & 1)) return;
-          tc_fence_after();
-          tmem_st32(lane_addr + pcol, v[0]);
+          tmem_st32(lane_addr + scol, v[0]);
+          tmem_st32(lane_addr + scol + 32, v[1]);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(p_full);
+          mbar_arrive(&p_full[s]);
         }
-        if (!wait_all(o_ready, oc & 1)) return;
+        if (!wait_all(&o_ready[s], oc & 1)) return;
         ++oc;
         tc_fence_after();
-        // the row sum is split between the two halves
-        red_sum[hf * kBlockM + r] = l;
-        mbar_arrive(xsum);
-        if (!wait_all(xsum, (oc - 1) & 1)) return;
-        const float lt = red_sum[kBlockM + r] + red_sum[r];
         const bool pad = i >= w.q_len;
-        const float inv = (lt > 0.f) ? 1.f / lt : __int_as_float(0x7fc00000);
+        const float inv = (l > 0.f) ? 1.f / l : __int_as_float(0x7fc00000);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(lane_addr + ocol + c * 32, o);
           tmem_wait_ld();
@@ -604,8 +653,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               uint32_t wv[4];
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const float a0 = pad ? 0.f : (lt > 0.f ? __uint_as_float(o[e + 2 * k]) * inv : inv);
-                const float a1 = pad ? 0.f : (lt > 0.f ? __uint_as_float(o[e + 2 * k + 1]) * inv : inv);
+                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k]) * inv : inv);
+                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k + 1]) * inv : inv);
                 wv[k] = std::is_same<T, __half>::value ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
               }
               *reinterpret_cast<uint4*>(orow + c * 32 + e) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -613,13 +662,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
         }
         tc_fence_before();
-        mbar_arrive(o_free);
-        // red_sum is written again only after the next unit's first max exchange, which both
-        // halves complete after their reads above
+        mbar_arrive(&o_free[s]);
       }
     }();
   }
-  if (warp == kMmaWarp) {
+  if (warp == 9) {
     // every MMA this CTA issued has completed before its TMEM is released (also on a timeout)
     if (elected) mma_commit(drain);
     __syncwarp();
@@ -628,7 +675,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
