@@ -40,6 +40,29 @@ bool make_map(CUtensorMap* m, const void* base, int dtype, int D, int heads, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The 16-bit bias as a 4-d tensor map (keys, queries, heads, batch) for the shared-memory bias
+// tiles: box = 64 keys x 128 queries, 128B swizzle. A broadcast head / batch dimension
+// (stride 0) becomes an extent-1 dimension read at coordinate 0. Needs the keys contiguous and
+// queries not broadcast; returns false otherwise (the kernel then reads the bias directly).
+bool make_bias_map(CUtensorMap* m, const Problem& P) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !P.bias || P.bias_dtype == SDPA_F32 || P.bs[0] != 1 || P.bs[1] <= 0) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)P.Lk, (cuuint64_t)P.Lq, (cuuint64_t)(P.bs[2] != 0 ? P.H : 1),
+                              (cuuint64_t)(P.bs[3] != 0 ? P.B : 1)};
+  // an extent-1 (broadcast) dimension gets the packed stride after the previous dimension
+  const long long row = P.bs[1] * 2;
+  const long long sh = P.bs[2] != 0 ? P.bs[2] * 2 : row * P.Lq;
+  const long long sb = P.bs[3] != 0 ? P.bs[3] * 2 : sh * (long long)dims[2];
+  if (row % 16 || sh % 16 || sb % 16 || row <= 0 || sh <= 0 || sb <= 0) return false;
+  const cuuint64_t strides[3] = {(cuuint64_t)row, (cuuint64_t)sh, (cuuint64_t)sb};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt = P.dtype == SDPA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(m, dt, 4, const_cast<void*>(P.bias), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int n = [] {
     int dev = 0, v = 0;
@@ -82,21 +105,22 @@ size_t prefill_workspace_bytes(const Problem&) { return 0; }
 
 cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const void* v, void* out, void*,
                            cudaStream_t stream, const char** msg) {
-  prefill::TensorMaps maps;
+  prefill::TensorMaps maps{};
   if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
       !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B)) {
     if (msg) *msg = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
+  const bool bias_tiles = P.D == 64 && make_bias_map(&maps.bias, P);
   const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
   const int grid = (int)std::min<long long>(n_units, sm_count());
   cudaError_t e;
   if (P.dtype == SDPA_BF16)
-    e = P.D == 128 ? prefill::launch<__nv_bfloat16, 128>(maps, P, out, grid, stream)
-                   : prefill::launch<__nv_bfloat16, 64>(maps, P, out, grid, stream);
+    e = P.D == 128 ? prefill::launch<__nv_bfloat16, 128>(maps, P, out, grid, false, stream)
+                   : prefill::launch<__nv_bfloat16, 64>(maps, P, out, grid, bias_tiles, stream);
   else
-    e = P.D == 128 ? prefill::launch<__half, 128>(maps, P, out, grid, stream)
-                   : prefill::launch<__half, 64>(maps, P, out, grid, stream);
+    e = P.D == 128 ? prefill::launch<__half, 128>(maps, P, out, grid, false, stream)
+                   : prefill::launch<__half, 64>(maps, P, out, grid, bias_tiles, stream);
   if (e != cudaSuccess && msg) *msg = "prefill launch";
   return e;
 }

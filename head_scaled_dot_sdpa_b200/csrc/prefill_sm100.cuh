@@ -64,7 +64,9 @@ constexpr int kUnitConsumers = 9;    // the MMA warp and the 8 softmax warps
 constexpr int kSchedWord = 16;       // int offset in the status area of the unit counter (+1: done)
 
 // bias / mask variants compiled into the kernel
-enum { kBiasNone = 0, kBiasSame = 1, kBiasF32 = 2 };
+// kBiasTile: a 16-bit bias brought into shared memory by TMA, one 128 x 128 tile per query tile
+// and key tile (head_dim 64, where the shared memory holds it); the others read global memory.
+enum { kBiasNone = 0, kBiasSame = 1, kBiasF32 = 2, kBiasTile = 3 };
 enum { kMaskNone = 0, kMaskDense = 1, kMaskBits = 2 };
 
 template <int D>
@@ -73,12 +75,19 @@ struct Cfg {
   static constexpr int kTileBytes = kRegions * kRegionBytes;
   static constexpr int kKStages = D == 128 ? 2 : 4;
   static constexpr int kVStages = D == 128 ? 2 : 4;
-  static constexpr int kBarriers = 2 * 2 + 2 * kKStages + 2 * kVStages + 2 * 4 + 1 + 2 * kUnitSlots;
-  static constexpr int kSmemBytes = (2 + kKStages + kVStages) * kTileBytes + kBarriers * 8 + 64 + 1024;
+  static constexpr int kBiasTileBytes = 128 * 128 * 2;
+  static constexpr int kBarriers = 2 * 2 + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 + 1 + 2 * kUnitSlots;
+  // tiles (+ one bias tile per query tile), barriers, unit ring, TMEM address, abort flag, and
+  // slack to align the base to 1024 bytes
+  static constexpr int smem_bytes(bool bias_tiles) {
+    return (2 + kKStages + kVStages) * kTileBytes + (bias_tiles ? 2 * kBiasTileBytes : 0) + kBarriers * 8 + 64 +
+           1024;
+  }
 };
+static_assert(Cfg<64>::smem_bytes(true) <= 227 * 1024, "bias tiles fit for head_dim 64");
 
 struct TensorMaps {
-  CUtensorMap q, k, v;
+  CUtensorMap q, k, v, bias;  // bias: (keys, queries, heads, batch), used by kBiasTile only
 };
 
 // One query tile of a unit.
@@ -200,7 +209,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint8_t* q_smem = smem;  // [2] tiles
   uint8_t* k_smem = q_smem + 2 * C::kTileBytes;
   uint8_t* v_smem = k_smem + C::kKStages * C::kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(v_smem + C::kVStages * C::kTileBytes);
+  uint8_t* b_smem = v_smem + C::kVStages * C::kTileBytes;  // [2] bias tiles (kBiasTile)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + (kBias == kBiasTile ? 2 * C::kBiasTileBytes : 0));
   uint64_t* q_full = bars;                  // [2]
   uint64_t* q_empty = q_full + 2;           // [2]
   uint64_t* k_full = q_empty + 2;           // [KS]
@@ -211,7 +221,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint64_t* p_full = s_full + 2;            // [2]
   uint64_t* o_ready = p_full + 2;           // [2]
   uint64_t* o_free = o_ready + 2;           // [2]
-  uint64_t* drain = o_free + 2;
+  uint64_t* b_full = o_free + 2;            // [2] bias tile of the stream loaded
+  uint64_t* b_empty = b_full + 2;           // [2] bias tile read by the stream's softmax
+  uint64_t* drain = b_empty + 2;
   uint64_t* unit_full = drain + 1;               // [kUnitSlots]
   uint64_t* unit_empty = unit_full + kUnitSlots; // [kUnitSlots]
   int* unit_ring = reinterpret_cast<int*>(unit_empty + kUnitSlots);
@@ -229,6 +241,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       mbar_init(&p_full[s], kBlockM);
       mbar_init(&o_ready[s], 1);
       mbar_init(&o_free[s], kBlockM);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], kBlockM);
     }
     for (int s = 0; s < C::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < C::kVStages; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
@@ -248,6 +262,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     prefetch_tmap(&maps.q);
     prefetch_tmap(&maps.k);
     prefetch_tmap(&maps.v);
+    if (kBias == kBiasTile) prefetch_tmap(&maps.bias);
   }
   tc_fence_before();
   __syncthreads();
@@ -286,6 +301,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     [&] {
       uint32_t g = 0;            // key tiles loaded so far (ring position)
       uint32_t qc[2] = {0, 0};   // Q tiles loaded per stream
+      uint32_t bc[2] = {0, 0};   // bias tiles loaded per stream
       // self-test: wait for a phase no one completes (the consumers' first release of slot 0)
       if (P.selftest_stall && !wait_all(&unit_empty[0], 0)) return;
       for (uint32_t k = 0;; ++k) {
@@ -339,6 +355,25 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               for (int r = 0; r < C::kRegions; ++r)
                 tma_load_4d(v_smem + vs * C::kTileBytes + r * kRegionBytes, &maps.v, &v_full[vs], r * 64,
                             w.kvh, prev_kb * kBlockN, w.b);
+            }
+          }
+          if constexpr (kBias == kBiasTile) {
+            // the bias tile (queries of the stream's tile x keys of kb), once the stream's
+            // softmax has read the previous one; broadcast dimensions use coordinate 0
+            if (kb != kNone) {
+#pragma unroll
+              for (int s = 0; s < 2; ++s) {
+                if ((s == 0 ? na : nb) != kb) continue;
+                if (!wait_all(&b_empty[s], (bc[s] & 1) ^ 1)) return;
+                if (elected) {
+                  mbar_arrive_expect_tx(&b_full[s], C::kBiasTileBytes);
+                  const int hb = P.bs[2] != 0 ? w.t[s].h : 0, bb = P.bs[3] != 0 ? w.b : 0;
+                  for (int r = 0; r < 2; ++r)
+                    tma_load_4d(b_smem + s * C::kBiasTileBytes + r * kRegionBytes, &maps.bias, &b_full[s],
+                                kb * kBlockN + r * 64, w.t[s].i0, hb, bb);
+                }
+                ++bc[s];
+              }
             }
           }
           __syncwarp();
@@ -464,7 +499,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
-      uint32_t sc = 0, oc = 0;
+      uint32_t sc = 0, oc = 0, bcs = 0;  // S tiles, units, bias tiles seen
       for (uint32_t kq = 0;; ++kq) {
         int u;
         if (!next_unit(kq, u)) return;
@@ -526,6 +561,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                                 (kMask == kMaskBits && (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu));
           const bool fast = kBias == kBiasNone && kMask != kMaskDense && __all_sync(0xffffffffu, full_row);
           float mul;
+          const uint8_t* bsm = b_smem + s * C::kBiasTileBytes;
+          if constexpr (kBias == kBiasTile) {
+            if (!wait_all(&b_full[s], bcs & 1)) return;
+          }
           if (fast) {
             mul = sl2;
 #pragma unroll
@@ -544,7 +583,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                 for (int e = 0; e < 32; e += 8) {
                   const int col = c * 32 + e;
                   float f8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                  if (col + 8 <= nvalid) {
+                  if constexpr (kBias == kBiasTile) {
+                    // 128-byte swizzled rows: 16-byte chunk ch of row r sits at chunk ch ^ (r % 8)
+                    const int box = col >> 6, ch = (col & 63) >> 3;
+                    load8<BT>(reinterpret_cast<const BT*>(bsm + box * kRegionBytes + r * 128 + ((ch ^ (r & 7)) << 4)), f8);
+                  } else if (col + 8 <= nvalid) {
                     load8<BT>(bias_row + key0 + col, f8);
                   } else {
 #pragma unroll
@@ -585,6 +628,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                 mx[e & 3] = fmaxf(mx[e & 3], t);
               }
             }
+          }
+          if constexpr (kBias == kBiasTile) {
+            mbar_arrive(&b_empty[s]);  // the bias tile has been read
+            ++bcs;
           }
           const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * mul;
           // the running max moves only when the row max passes it by 2^8 (or leaves -inf)
@@ -690,18 +737,20 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   }
 }
 
-// Host launcher for one (T, D) pair; defined in the per-type translation units.
+// Host launcher for one (T, D) pair; defined in the per-type translation units. bias_tiles:
+// maps.bias describes the bias and the kBiasTile variant may be used (head_dim 64 only).
 template <typename T, int D>
-cudaError_t launch(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream);
-template <> cudaError_t launch<__nv_bfloat16, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
-template <> cudaError_t launch<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
-template <> cudaError_t launch<__half, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
-template <> cudaError_t launch<__half, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+cudaError_t launch(const TensorMaps& maps, const Problem& P, void* out, int grid, bool bias_tiles,
+                   cudaStream_t stream);
+template <> cudaError_t launch<__nv_bfloat16, 128>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
+template <> cudaError_t launch<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
+template <> cudaError_t launch<__half, 128>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
+template <> cudaError_t launch<__half, 64>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
 
 template <typename T, int D, int kBias, int kMask>
 cudaError_t launch_variant(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream) {
   auto kern = prefill_kernel<T, D, kBias, kMask>;
-  const int smem = Cfg<D>::kSmemBytes;
+  const int smem = Cfg<D>::smem_bytes(kBias == kBiasTile);
   // checked and configured once per device (bit d of `ready`)
   static std::atomic<unsigned long long> ready{0};
   int dev = 0;
@@ -723,9 +772,10 @@ cudaError_t launch_variant(const TensorMaps& maps, const Problem& P, void* out, 
   return cudaGetLastError();
 }
 
-inline int bias_variant(const Problem& P) {
+inline int bias_variant(const Problem& P, bool bias_tiles) {
   if (!P.bias) return kBiasNone;
-  return P.bias_dtype == SDPA_F32 ? kBiasF32 : kBiasSame;
+  if (P.bias_dtype == SDPA_F32) return kBiasF32;
+  return bias_tiles ? kBiasTile : kBiasSame;
 }
 inline int mask_variant(const Problem& P) {
   if (P.bcls) return kMaskBits;
@@ -736,8 +786,15 @@ inline int mask_variant(const Problem& P) {
 #define SDPA_PREFILL_DEFINE_LAUNCH(T, D)                                                              \
   template <>                                                                                       \
   cudaError_t launch<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,         \
-                           cudaStream_t stream) {                                                   \
-    const int b = bias_variant(P), m = mask_variant(P);                                             \
+                           bool bias_tiles, cudaStream_t stream) {                                  \
+    const int b = bias_variant(P, bias_tiles && D == 64), m = mask_variant(P);                      \
+    if constexpr (D == 64) {                                                                        \
+      if (b == kBiasTile) {                                                                         \
+        if (m == kMaskNone) return launch_variant<T, D, kBiasTile, kMaskNone>(maps, P, out, grid, stream); \
+        if (m == kMaskDense) return launch_variant<T, D, kBiasTile, kMaskDense>(maps, P, out, grid, stream); \
+        return launch_variant<T, D, kBiasTile, kMaskBits>(maps, P, out, grid, stream);              \
+      }                                                                                             \
+    }                                                                                               \
     switch (b * 3 + m) {                                                                            \
       case 0: return launch_variant<T, D, kBiasNone, kMaskNone>(maps, P, out, grid, stream);        \
       case 1: return launch_variant<T, D, kBiasNone, kMaskDense>(maps, P, out, grid, stream);       \

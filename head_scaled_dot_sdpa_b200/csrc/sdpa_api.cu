@@ -273,6 +273,8 @@ sdpa_status build_block_mask_info(const uint8_t* mask, const int64_t mask_stride
     return fail(SDPA_ERR_WORKSPACE, "info buffer must be non-NULL and 256-byte aligned");
   if (info_bytes < need) return fail(SDPA_ERR_WORKSPACE, "info buffer has %zu bytes, needs %zu", info_bytes, need);
   const int nqb = (q_len + bq - 1) / bq, nkb = (kv_len + bk - 1) / bk;
+  if (nqb > 65535 || nheads > 65535)
+    return fail(SDPA_ERR_INVALID_ARG, "at most 65535 query blocks and 65535 mask heads (got %d, %d)", nqb, nheads);
   const size_t blocks = (size_t)nheads * nqb * nkb;
   char* base = static_cast<char*>(info_buf);
   uint8_t* cls = reinterpret_cast<uint8_t*>(base);

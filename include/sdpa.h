@@ -212,7 +212,9 @@ SDPA_API size_t build_block_mask_info_size(int32_t nheads, int32_t q_len, int32_
  * must be 1) as empty, partial or full, packs the bits of the partial blocks and lists the
  * non-empty blocks of every block row (see sdpa_block_mask_info). The result lives in the
  * caller's `info_buf` and is described by *out_info, filled in on the host before return.
- * sdpa_forward uses it when bq = bk = 128. */
+ * sdpa_forward uses it when bq = bk = 128. At most 65535 query blocks and 65535 mask heads
+ * (SDPA_ERR_INVALID_ARG beyond). Two kernels run on `stream`: one per block, then one that
+ * builds the block-row lists. */
 SDPA_API sdpa_status build_block_mask_info(const uint8_t* mask, const int64_t mask_stride[3],
                                   int32_t nheads, int32_t q_len, int32_t kv_len, int32_t bq,
                                   int32_t bk, void* info_buf, size_t info_bytes,

@@ -89,6 +89,32 @@ def test_prefill_bias_and_mask(bias_dtype):
     assert_matches(out, want, 1e-2, "bias+mask")
 
 
+BIAS_LAYOUTS = {
+    # shape of the bias tensor, broadcast to (B, H, Lq, Lk)
+    "bhqk": lambda B, H, Lq, Lk: (B, H, Lq, Lk),
+    "qk": lambda B, H, Lq, Lk: (Lq, Lk),          # shared by every batch element and head
+    "b1qk": lambda B, H, Lq, Lk: (B, 1, Lq, Lk),  # shared by the heads
+    "hk": lambda B, H, Lq, Lk: (H, 1, Lk),        # one row per head, shared by the queries
+}
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("layout", list(BIAS_LAYOUTS))
+@pytest.mark.parametrize("causal", [False, True])
+def test_prefill_bias_layouts(D, layout, causal):
+    # 272 keys: 16-byte aligned rows; 300 queries: three query tiles (one unit with one tile)
+    B, Lq, Lk, H, Hkv = 2, 300, 272, 4, 2
+    rng = _rng(11 + D)
+    q, k, v = _qkv(12 + D, B, Lq, Lk, H, Hkv, D, torch.bfloat16)
+    # unit-variance bias (ALiBi / T5 magnitudes): a near one-hot softmax would put outputs of
+    # |v| ~ 3 on the bf16 grid, whose half-spacing there (0.0078) alone nearly fills 1e-2
+    bias = torch.from_numpy(rng.standard_normal(BIAS_LAYOUTS[layout](B, H, Lq, Lk)).astype(np.float32))
+    bias = bias.to(torch.bfloat16)
+    out = run(q, k, v, bias.to(DEV), is_causal=causal)
+    want = oracle.sdpa_forward(f64(q), f64(k), f64(v), bias=f64(bias), is_causal=causal)
+    assert_matches(out, want, 1e-2, f"bias {layout} D={D}")
+
+
 def test_prefill_block_info():
     w = si.scaled(si.BLOCK_SPARSE, nheads=4, q_len=600, kv_len=900, block=128)
     cls = si.block_classes(w)
