@@ -10,14 +10,15 @@
 // kv_lengths prefix, or the non-empty blocks of a block-sparse mask), each loaded once.
 //
 // Warp roles (384 threads):
-//   warp 8      TMA producer: Q_A, Q_B, then K_u ahead of V_{u-1} through 128B-swizzled rings;
-//   warp 9      MMA issuer and TMEM owner (warps 10-11 idle; warpgroup 2 gives its registers to
-//               the softmax warpgroups with setmaxnreg). Per key tile u, in this order:
-//                 O_A += P_A(u-1) V(u-1);  S_A(u) = Q_A K(u)^T;
-//                 O_B += P_B(u-1) V(u-1);  S_B(u) = Q_B K(u)^T
-//               (S: tcgen05.mma with both operands in shared memory; PV: P read from TMEM). So
-//               the tensor pipe works on one tile while the other tile's softmax runs, and the
-//               in-order tcgen05 pipeline lets S_X(u) reuse the columns PV_X(u-1) just read;
+//   warp 8      TMA producer: Q_A, Q_B, then K_u ahead of V_{u-1} (and the bias tiles of the
+//               shared-memory bias variant) through 128B-swizzled rings;
+//   warps 9, 11 MMA issuers of tile A and tile B (warp 9 owns the TMEM; warp 10 idle;
+//               warpgroup 2 gives its registers to the softmax warpgroups with setmaxnreg).
+//               Per key tile u each issues O_X += P_X(u-1) V(u-1); S_X(u) = Q_X K(u)^T (S:
+//               both operands in shared memory; PV: P read from TMEM; the in-order tcgen05
+//               pipeline lets S_X(u) reuse the columns PV_X(u-1) just read). A turn order
+//               between the two warps keeps the issue order A, B, A, B, so the tensor pipe
+//               works on one tile while the other tile's softmax runs;
 //   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: one thread per query row
 //               (= TMEM lane). tcgen05.ld of the S row; masks (causal / q_offset / kv_lengths
 //               as one prefix bound per row, boolean mask bytes or partial-block bits); optional
@@ -60,7 +61,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 bytes (64 16-bit columns)
 constexpr int kNone = 1 << 30;
 constexpr int kUnitSlots = 4;        // ring of unit indices handed from the producer to the others
-constexpr int kUnitConsumers = 9;    // the MMA warp and the 8 softmax warps
+constexpr int kUnitConsumers = 10;   // the two MMA warps and the 8 softmax warps
+constexpr int kMmaWarpA = 9, kMmaWarpB = 11;  // MMA issuers of tile A and tile B
 constexpr int kSchedWord = 16;       // int offset in the status area of the unit counter (+1: done)
 
 // bias / mask variants compiled into the kernel
@@ -229,6 +231,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   int* unit_ring = reinterpret_cast<int*>(unit_empty + kUnitSlots);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring + kUnitSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // MMA groups issued so far by the MMA warp of tile A / tile B (the turn order below)
+  volatile uint32_t* issued = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);  // [2]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint64_t tmo = P.wait_timeout_ns;
@@ -244,17 +248,20 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], kBlockM);
     }
-    for (int s = 0; s < C::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-    for (int s = 0; s < C::kVStages; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
-    mbar_init(drain, 1);
+    // a K / V slot is released by both MMA warps
+    for (int s = 0; s < C::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 2); }
+    for (int s = 0; s < C::kVStages; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 2); }
+    mbar_init(drain, 2);
     for (int k = 0; k < kUnitSlots; ++k) {
       mbar_init(&unit_full[k], 1);
       mbar_init(&unit_empty[k], kUnitConsumers);
     }
     *abort_flag = 0;
+    issued[0] = 0;
+    issued[1] = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarpA) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -385,38 +392,73 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         }
       }
     }();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarpA || warp == kMmaWarpB) {
+    // ------------------------------------------------------------------ MMA issuers
+    // One warp per query tile, so that each tile's PV and next S are issued as soon as its
+    // own P is ready, whatever the other tile is doing. Both walk the union of the two key
+    // lists in the same order; each releases every K / V slot once: by a commit after its
+    // last MMA on the slot, or, for a key tile it does not visit, by an arrive once the slot
+    // holds that tile (so the arrive always counts toward the slot's current phase).
     [&] {
+      const int s = warp == kMmaWarpA ? 0 : 1;
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_qk = instr_desc_f16(kBf16, false, false, kBlockM, kBlockN);
       constexpr uint32_t idesc_pv = instr_desc_f16(kBf16, false, true, kBlockM, D);
-      const uint32_t q_base = smem_addr(q_smem), k_base = smem_addr(k_smem), v_base = smem_addr(v_smem);
-      uint32_t g = 0;
-      uint32_t sc[2] = {0, 0};  // S tiles issued per stream (phase of s_full / p_full)
-      uint32_t qc[2] = {0, 0};
-      uint32_t oc[2] = {0, 0};  // units per stream (phase of o_ready / o_free)
+      const uint32_t qtile = smem_addr(q_smem) + s * C::kTileBytes;
+      const uint32_t k_base = smem_addr(k_smem), v_base = smem_addr(v_smem);
+      const uint32_t s_tmem = tmem + s * 128, o_tmem = tmem + 256 + s * D;
+      // Turn order. A tile's MMAs come in groups: S(0); PV(j-1) + S(j); the last PV. Group k
+      // of tile A follows group k-1 of tile B, and group k of B follows group k of A, as a
+      // single issuer would order them, so the two softmaxes stay half a period apart.
+      // Only used when one key list is a prefix of the other (no block list): then neither
+      // warp can wait on a K / V slot the other has yet to release.
+      const bool turns = P.bcls == nullptr;
+      uint32_t base_o = 0;        // groups the other tile issued before this unit
+      uint32_t mine = 0;          // groups this warp has issued in total
+      auto turn_wait = [&](uint32_t target) -> bool {
+        if (!turns || issued[s ^ 1] >= target) return true;
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t n = 1;; ++n) {
+          if (issued[s ^ 1] >= target) return true;
+          if ((n & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > tmo) {
+              fail();
+              return false;
+            }
+          }
+        }
+      };
+      auto published = [&]() {
+        __syncwarp();
+        ++mine;
+        if (elected) issued[s] = mine;
+        __syncwarp();
+      };
+      uint32_t g = 0, sc = 0, qc = 0, oc = 0;
       for (uint32_t kq = 0;; ++kq) {
         int u;
         if (!next_unit(kq, u)) return;
         if (u >= n_units) break;
         const Unit w = make_unit(P, u);
         if (w.t[0].n == 0 && w.t[1].n == 0) continue;
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          if (w.t[s].n == 0) continue;
-          if (!wait_all(&q_full[s], qc[s] & 1)) return;
-          ++qc[s];
+        // (selects on scalars only: an index that depends on the warp would put the unit in
+        // local memory)
+        const int my_n = s == 0 ? w.t[0].n : w.t[1].n;
+        const int n_o = s == 0 ? w.t[1].n : w.t[0].n;
+        const uint32_t groups_o = n_o > 0 ? (uint32_t)n_o + 1 : 0u;
+        // group k of this tile may be issued once the other tile has issued `before(k)` groups
+        auto before = [&](uint32_t k) -> uint32_t { return base_o + min(s == 0 ? k : k + 1, groups_o); };
+        if (my_n > 0) {
+          if (!wait_all(&q_full[s], qc & 1)) return;
+          ++qc;
         }
-        bool pend[2] = {false, false};  // a PV of the previous key tile is owed
-        bool first_pv[2] = {true, true};
-        int ja = 0, jb = 0;
-        // PV of stream s for the key tile at ring position x (waits for its P)
-        auto pv = [&](int s, uint32_t x) -> bool {
-          if (!wait_all(&p_full[s], (sc[s] - 1) & 1)) return false;
+        // O += P(x) V(x) for this tile's key tile at ring position x (waits for its P)
+        auto pv = [&](uint32_t x, bool first) -> bool {
+          if (!wait_all(&p_full[s], (sc - 1) & 1)) return false;
           const int vs = x % C::kVStages;
           if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
-          if (first_pv[s] && !wait_all(&o_free[s], (oc[s] & 1) ^ 1)) return false;
+          if (first && !wait_all(&o_free[s], (oc & 1) ^ 1)) return false;
           tc_fence_after();
           if (elected) {
             const uint32_t vtile = v_base + vs * C::kTileBytes;
@@ -425,69 +467,84 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               // B = V (keys x dims, dims contiguous): MN-major; 64-dim regions kRegionBytes
               // apart (LBO), 8-key groups 1024 bytes apart (SBO); 16 keys per step.
               const uint64_t bdesc = smem_desc_sw128(vtile + kk * 16 * 128, kRegionBytes, 1024);
-              mma_ts(tmem + 256 + s * D, tmem + s * 128 + kk * 8, bdesc, idesc_pv,
-                     (first_pv[s] && kk == 0) ? 0u : 1u);
+              mma_ts(o_tmem, s_tmem + kk * 8, bdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
             }
+            mma_commit(&v_empty[vs]);
           }
           __syncwarp();
-          first_pv[s] = false;
           return true;
         };
-        auto qk = [&](int s, int ks) {
-          tc_fence_after();
-          if (elected) {
-            const uint32_t qtile = q_base + s * C::kTileBytes, ktile = k_base + ks * C::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              // A = Q, B = K: both K-major, 128-byte rows, 8-row groups 1024 bytes apart.
-              const uint32_t off = (kk / 4) * kRegionBytes + (kk % 4) * 32;
-              mma_ss(tmem + s * 128, smem_desc_sw128(qtile + off, 16, 1024),
-                     smem_desc_sw128(ktile + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&s_full[s]);
-          }
-          __syncwarp();
-          ++sc[s];
-        };
+        int ja = 0, jb = 0, jm = 0;
+        uint32_t k_grp = 0;  // groups of this tile issued in this unit
+        bool pend = false, first_pv = true;
+        uint32_t prev = 0;
         for (;;) {
           const int na = w.t[0].next(ja), nb = w.t[1].next(jb);
           const int kb = min(na, nb);
-          const bool in[2] = {kb != kNone && na == kb, kb != kNone && nb == kb};
-          const uint32_t x = g;  // ring position of this key tile
-          const int ks = x % C::kKStages;
-          if (kb != kNone && !wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
-  #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            if (pend[s] && !pv(s, x - 1)) return;
-            if (in[s]) {
-              qk(s, ks);
-              // the stream's last S has been issued: Q_s may be reloaded once it completes
-              if (elected && (s == 0 ? ja : jb) + 1 == w.t[s].n) mma_commit(&q_empty[s]);
-            }
-          }
-          if (elected) {
-            if (pend[0] || pend[1]) mma_commit(&v_empty[(x - 1) % C::kVStages]);
-            if (kb != kNone) mma_commit(&k_empty[ks]);
-          }
-          __syncwarp();
           if (kb == kNone) break;
-          pend[0] = in[0];
-          pend[1] = in[1];
-          if (in[0]) ++ja;
-          if (in[1]) ++jb;
+          const bool mine_tile = (s == 0 ? na : nb) == kb;
+          const uint32_t x = g;
+          const int ks = x % C::kKStages, vs = x % C::kVStages;
+          if (!mine_tile) {
+            // a key tile only the other query tile visits: first the PV this tile owes (its
+            // V slot may be needed before this warp reaches its next own key tile), then
+            // release the slots once they hold this key tile
+            if (pend) {
+              if (!turn_wait(before(k_grp))) return;
+              if (!pv(prev, first_pv)) return;
+              published();
+              ++k_grp;
+              first_pv = false;
+              pend = false;
+            }
+            if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
+            if (elected) mbar_arrive(&k_empty[ks]);
+            if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return;
+            if (elected) mbar_arrive(&v_empty[vs]);
+          } else {
+            if (!turn_wait(before(k_grp))) return;
+            // PV of this tile's previous key tile first: S(x) overwrites the P it reads
+            if (pend && !pv(prev, first_pv)) return;
+            if (pend) first_pv = false;
+            if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
+            tc_fence_after();
+            if (elected) {
+              const uint32_t ktile = k_base + ks * C::kTileBytes;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                // A = Q, B = K: both K-major, 128-byte rows, 8-row groups 1024 bytes apart.
+                const uint32_t off = (kk / 4) * kRegionBytes + (kk % 4) * 32;
+                mma_ss(s_tmem, smem_desc_sw128(qtile + off, 16, 1024), smem_desc_sw128(ktile + off, 16, 1024),
+                       idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(&s_full[s]);
+              mma_commit(&k_empty[ks]);
+              // the tile's last S: Q may be reloaded once it completes
+              if (jm + 1 == my_n) mma_commit(&q_empty[s]);
+            }
+            published();
+            ++k_grp;
+            ++sc;
+            ++jm;
+            pend = true;
+            prev = x;
+          }
+          if (na == kb) ++ja;
+          if (nb == kb) ++jb;
           ++g;
         }
-        if (elected) {
-  #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            if (w.t[s].n == 0) continue;
-            mma_commit(&o_ready[s]);
-          }
+        if (pend) {
+          if (!turn_wait(before(k_grp))) return;
+          if (!pv(prev, first_pv)) return;
+          published();
+          ++k_grp;
         }
-        __syncwarp();
-#pragma unroll
-        for (int s = 0; s < 2; ++s)
-          if (w.t[s].n != 0) ++oc[s];
+        if (my_n > 0) {
+          if (elected) mma_commit(&o_ready[s]);
+          __syncwarp();
+          ++oc;
+        }
+        base_o += groups_o;
       }
     }();
   } else if (warp < 8) {
@@ -713,7 +770,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       }
     }();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarpA || warp == kMmaWarpB) {
     // every MMA this CTA issued has completed before its TMEM is released (also on a timeout)
     if (elected) mma_commit(drain);
     __syncwarp();
@@ -722,7 +779,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarpA) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
