@@ -281,7 +281,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     report(P.status, SDPA_ERR_TIMEOUT);
   };
   // every lane of a warp takes the same branch; a timeout seen by any lane stops the warp
+  // (A phase that has already completed is the common case: one try_wait and a vote settle it
+  // without the divergent polling loop, whose reconvergence costs tens of cycles.)
   auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     const bool ok = mbar_wait(bar, parity, tmo, abort_flag);
     if (__all_sync(0xffffffffu, ok)) return true;
     fail();
@@ -453,12 +456,17 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           if (!wait_all(&q_full[s], qc & 1)) return;
           ++qc;
         }
+        // V(x) loaded and, for the unit's first PV, O free: waited for ahead of the turn, so
+        // that they are off the path from "P ready" to the MMA issue
+        auto pv_ready = [&](uint32_t x, bool first) -> bool {
+          const int vs = x % C::kVStages;
+          if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
+          return !first || wait_all(&o_free[s], (oc & 1) ^ 1);
+        };
         // O += P(x) V(x) for this tile's key tile at ring position x (waits for its P)
         auto pv = [&](uint32_t x, bool first) -> bool {
           if (!wait_all(&p_full[s], (sc - 1) & 1)) return false;
           const int vs = x % C::kVStages;
-          if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
-          if (first && !wait_all(&o_free[s], (oc & 1) ^ 1)) return false;
           tc_fence_after();
           if (elected) {
             const uint32_t vtile = v_base + vs * C::kTileBytes;
@@ -490,6 +498,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             // V slot may be needed before this warp reaches its next own key tile), then
             // release the slots once they hold this key tile
             if (pend) {
+              if (!pv_ready(prev, first_pv)) return;
               if (!turn_wait(before(k_grp))) return;
               if (!pv(prev, first_pv)) return;
               published();
@@ -502,11 +511,12 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return;
             if (elected) mbar_arrive(&v_empty[vs]);
           } else {
+            if (pend && !pv_ready(prev, first_pv)) return;
+            if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
             if (!turn_wait(before(k_grp))) return;
             // PV of this tile's previous key tile first: S(x) overwrites the P it reads
             if (pend && !pv(prev, first_pv)) return;
             if (pend) first_pv = false;
-            if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
             tc_fence_after();
             if (elected) {
               const uint32_t ktile = k_base + ks * C::kTileBytes;
@@ -534,6 +544,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           ++g;
         }
         if (pend) {
+          if (!pv_ready(prev, first_pv)) return;
           if (!turn_wait(before(k_grp))) return;
           if (!pv(prev, first_pv)) return;
           published();
