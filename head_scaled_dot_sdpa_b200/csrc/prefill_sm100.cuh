@@ -201,6 +201,22 @@ __device__ __forceinline__ void load8(const BT* p, float (&f)[8]) {
   }
 }
 
+// O (D fp32 columns of this thread's TMEM lane) *= a. Rare (the running max moved by more
+// than 2^8), so it is kept out of line: its code and registers stay off the softmax loop.
+template <int D>
+__device__ __noinline__ void rescale_o(uint32_t taddr, float a) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(taddr + c * 32, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
+    tmem_st32(taddr + c * 32, o);
+  }
+  tmem_wait_st();
+}
+
 template <typename T, int D, int kBias, int kMask>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __restrict__ out, int n_units) {
@@ -633,8 +649,20 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           if constexpr (kBias == kBiasTile) {
             if (!wait_all(&b_full[s], bcs & 1)) return;
           }
-          if (fast) {
+          if (kBias == kBiasNone && kMask != kMaskDense) {
+            // No bias: the raw scores stay raw (the max commutes with scale > 0) and a masked
+            // key only has to become -inf; one keep-word per 32 keys drives the selects.
             mul = sl2;
+            if (!fast) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int lim = nvalid - 32 * c;
+                uint32_t keep = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
+                if constexpr (kMask == kMaskBits) keep &= bw[c];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[c][e] = ((keep >> e) & 1u) ? v[c][e] : 0xff800000u;
+              }
+            }
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -713,20 +741,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             m_used = rmax;
           }
           const bool need_o = grow && had_max && j > 0;
-          if (__any_sync(0xffffffffu, need_o)) {
-            // O holds PV of the earlier key tiles (complete: the S commit covered them)
-            const float a = need_o ? alpha : 1.f;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(lane_addr + ocol + c * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
-              tmem_st32(lane_addr + ocol + c * 32, o);
-            }
-            tmem_wait_st();
-          }
+          // O holds PV of the earlier key tiles (complete: the S commit covered them)
+          if (__any_sync(0xffffffffu, need_o)) rescale_o<D>(lane_addr + ocol, need_o ? alpha : 1.f);
           l *= alpha;
           const float negm = (m_used == -INFINITY) ? 0.f : -m_used;
           // P = 2^(v * mul - m), 16-bit pairs into the first 64 columns of the tile's S columns.
