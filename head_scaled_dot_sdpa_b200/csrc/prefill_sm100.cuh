@@ -448,12 +448,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
         }
       };
-      auto published = [&]() {
-        __syncwarp();
-        ++mine;
-        if (elected) issued[s] = mine;
-        __syncwarp();
-      };
+      // the elected lane publishes a group as soon as its last MMA is issued (before the
+      // commits): the other warp may then queue its own group behind it
+      auto publish = [&]() { issued[s] = mine + 1; };
       uint32_t g = 0, sc = 0, qc = 0, oc = 0;
       for (uint32_t kq = 0;; ++kq) {
         int u;
@@ -474,14 +471,17 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         }
         // V(x) loaded and, for the unit's first PV, O free: waited for ahead of the turn, so
         // that they are off the path from "P ready" to the MMA issue
+        // (and P(x) written: usually long before the turn comes, so that the turn is the last
+        // wait before the MMAs)
         auto pv_ready = [&](uint32_t x, bool first) -> bool {
           const int vs = x % C::kVStages;
           if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
-          return !first || wait_all(&o_free[s], (oc & 1) ^ 1);
+          if (first && !wait_all(&o_free[s], (oc & 1) ^ 1)) return false;
+          return wait_all(&p_full[s], (sc - 1) & 1);
         };
-        // O += P(x) V(x) for this tile's key tile at ring position x (waits for its P)
-        auto pv = [&](uint32_t x, bool first) -> bool {
-          if (!wait_all(&p_full[s], (sc - 1) & 1)) return false;
+        // O += P(x) V(x) for this tile's key tile at ring position x (after pv_ready); `last`:
+        // the group ends here and is published
+        auto pv = [&](uint32_t x, bool first, bool last) {
           const int vs = x % C::kVStages;
           tc_fence_after();
           if (elected) {
@@ -493,10 +493,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               const uint64_t bdesc = smem_desc_sw128(vtile + kk * 16 * 128, kRegionBytes, 1024);
               mma_ts(o_tmem, s_tmem + kk * 8, bdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
             }
+            if (last) publish();
             mma_commit(&v_empty[vs]);
           }
           __syncwarp();
-          return true;
         };
         int ja = 0, jb = 0, jm = 0;
         uint32_t k_grp = 0;  // groups of this tile issued in this unit
@@ -516,8 +516,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if (pend) {
               if (!pv_ready(prev, first_pv)) return;
               if (!turn_wait(before(k_grp))) return;
-              if (!pv(prev, first_pv)) return;
-              published();
+              pv(prev, first_pv, true);
+              ++mine;
               ++k_grp;
               first_pv = false;
               pend = false;
@@ -531,7 +531,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
             if (!turn_wait(before(k_grp))) return;
             // PV of this tile's previous key tile first: S(x) overwrites the P it reads
-            if (pend && !pv(prev, first_pv)) return;
+            if (pend) pv(prev, first_pv, false);
             if (pend) first_pv = false;
             tc_fence_after();
             if (elected) {
@@ -543,12 +543,14 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                 mma_ss(s_tmem, smem_desc_sw128(qtile + off, 16, 1024), smem_desc_sw128(ktile + off, 16, 1024),
                        idesc_qk, kk > 0 ? 1u : 0u);
               }
+              publish();
               mma_commit(&s_full[s]);
               mma_commit(&k_empty[ks]);
               // the tile's last S: Q may be reloaded once it completes
               if (jm + 1 == my_n) mma_commit(&q_empty[s]);
             }
-            published();
+            __syncwarp();
+            ++mine;
             ++k_grp;
             ++sc;
             ++jm;
@@ -562,8 +564,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if (pend) {
           if (!pv_ready(prev, first_pv)) return;
           if (!turn_wait(before(k_grp))) return;
-          if (!pv(prev, first_pv)) return;
-          published();
+          pv(prev, first_pv, true);
+          ++mine;
           ++k_grp;
         }
         if (my_n > 0) {
