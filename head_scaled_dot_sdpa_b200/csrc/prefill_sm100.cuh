@@ -258,9 +258,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], kBlockM);
+      mbar_init(&p_full[s], 4);  // one arrive per softmax warp
       mbar_init(&o_ready[s], 1);
-      mbar_init(&o_free[s], kBlockM);
+      mbar_init(&o_free[s], 4);
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], kBlockM);
     }
@@ -527,8 +527,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return;
             if (elected) mbar_arrive(&v_empty[vs]);
           } else {
-            if (pend && !pv_ready(prev, first_pv)) return;
             if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
+            if (pend && !pv_ready(prev, first_pv)) return;
             if (!turn_wait(before(k_grp))) return;
             // PV of this tile's previous key tile first: S(x) overwrites the P it reads
             if (pend) pv(prev, first_pv, false);
@@ -768,7 +768,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           tmem_st32(lane_addr + scol + 32, v[1]);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&p_full[s]);
+          __syncwarp();  // the warp's stores are done (each lane waited for its own)
+          if (lane == 0) mbar_arrive(&p_full[s]);
         }
         if (!wait_all(&o_ready[s], oc & 1)) return;
         ++oc;
@@ -795,7 +796,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
         }
         tc_fence_before();
-        mbar_arrive(&o_free[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[s]);
       }
     }();
   }
