@@ -315,7 +315,9 @@ decode_split_kernel(Problem P, const T* __restrict__ q, const T* __restrict__ kc
   }
 }
 
-// One warp per output row (b, t, h): merge the row's splits and normalise.
+// One warp per output row (b, t, h): merge the row's splits and normalise. Lane j holds the
+// (m, l) of splits j, j + 32, ... so the maximum and the weights come from shuffles, and the
+// partial O rows are then read with no dependence on a branch.
 template <typename T, int D>
 __global__ void decode_combine_kernel(Problem P, Partials part, T* __restrict__ out) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -332,22 +334,36 @@ __global__ void decode_combine_kernel(Problem P, Partials part, T* __restrict__ 
   const int kvh = h / P.group, r = t * P.group + (h % P.group);
   const long long pbase = ((long long)b * P.Hkv + kvh) * part.max_splits;
   float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, part.ml[((pbase + s) * kRows + r) * 2]);
+  for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, part.ml[((pbase + s) * kRows + r) * 2]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   constexpr int kPer = D / 32;
   float o[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) o[u] = 0.f;
   float L = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < n_splits; ++s) {
-      const long long pr = (pbase + s) * kRows + r;
-      const float ms = part.ml[pr * 2];
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L += f * part.ml[pr * 2 + 1];
+    for (int s0 = 0; s0 < n_splits; s0 += 32) {
+      // weight of split s0 + lane
+      float f = 0.f, lw = 0.f;
+      if (s0 + lane < n_splits) {
+        const long long pr = (pbase + s0 + lane) * kRows + r;
+        const float ms = part.ml[pr * 2];
+        f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        lw = f * part.ml[pr * 2 + 1];
+      }
+      L += lw;
+      const int n = min(32, n_splits - s0);
+#pragma unroll 4
+      for (int j = 0; j < n; ++j) {
+        const float fj = __shfl_sync(0xffffffffu, f, j);
+        const float* po = part.o + ((pbase + s0 + j) * kRows + r) * D + lane;
 #pragma unroll
-      for (int u = 0; u < kPer; ++u) o[u] += f * part.o[pr * D + lane + 32 * u];
+        for (int u = 0; u < kPer; ++u) o[u] += fj * po[32 * u];
+      }
     }
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
   }
   T* orow = out + row * D;
   const float inv = (L > 0.f) ? 1.f / L : __int_as_float(0x7fc00000);  // no key: NaN
@@ -355,9 +371,25 @@ __global__ void decode_combine_kernel(Problem P, Partials part, T* __restrict__ 
   for (int u = 0; u < kPer; ++u) orow[lane + 32 * u] = from_f32<T>(L > 0.f ? o[u] * inv : inv);
 }
 
+int sm_count() {
+  static int n = [] {
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v > 0 ? v : 148;
+  }();
+  return n;
+}
+
+// Keys per split: long splits stream longer and leave fewer partials to combine, but the grid
+// must still fill the GPU. The largest of 1024 / 512 / 256 keys that gives at least eight
+// CTAs per SM over the cache capacity (the lengths themselves are on the device).
 int pick_split(const Problem& P) {
-  (void)P;
-  return 512;
+  const long long pairs = (long long)P.B * P.Hkv;
+  for (int split : {1024, 512}) {
+    if (pairs * ((P.Lk + split - 1) / split) >= 8LL * sm_count()) return split;
+  }
+  return 256;
 }
 
 }  // namespace
