@@ -344,6 +344,16 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if (u >= n_units) break;
         const Unit w = make_unit(P, u);
         if (w.t[0].n == 0 && w.t[1].n == 0) continue;
+        // The unit's Q tiles come from DRAM (each is read once); their slots free only when
+        // the previous unit's last S completes, so they are first brought into L2 now, about
+        // two key tiles before that.
+        if (elected) {
+#pragma unroll
+          for (int s = 0; s < 2; ++s)
+            if (w.t[s].n > 0)
+              for (int r = 0; r < C::kRegions; ++r) tma_prefetch_l2_4d(&maps.q, r * 64, w.t[s].h, w.t[s].i0, w.b);
+        }
+        __syncwarp();
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           if (w.t[s].n == 0) continue;

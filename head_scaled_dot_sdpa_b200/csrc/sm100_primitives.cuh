@@ -73,6 +73,13 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, uint64_
       "r"(smem_addr(bar))
       : "memory");
 }
+// Brings the 4-d tile at the given coordinates from global memory into L2 (no shared memory,
+// no completion to wait for): a later tma_load_4d of the same tile then hits L2.
+__device__ __forceinline__ void tma_prefetch_l2_4d(const void* tmap, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];\n" ::"l"(tmap),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
