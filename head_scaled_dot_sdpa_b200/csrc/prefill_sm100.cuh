@@ -11,14 +11,16 @@
 //
 // Warp roles (384 threads):
 //   warp 8      TMA producer: Q_A, Q_B, then K_u ahead of V_{u-1} (and the bias tiles of the
-//               shared-memory bias variant) through 128B-swizzled rings;
+//               shared-memory bias variant) through 128B-swizzled rings; it also takes the units
+//               from the counter and prefetches their Q tiles into L2;
 //   warps 9, 11 MMA issuers of tile A and tile B (warp 9 owns the TMEM; warp 10 idle;
 //               warpgroup 2 gives its registers to the softmax warpgroups with setmaxnreg).
 //               Per key tile u each issues O_X += P_X(u-1) V(u-1); S_X(u) = Q_X K(u)^T (S:
 //               both operands in shared memory; PV: P read from TMEM; the in-order tcgen05
 //               pipeline lets S_X(u) reuse the columns PV_X(u-1) just read). A turn order
 //               between the two warps keeps the issue order A, B, A, B, so the tensor pipe
-//               works on one tile while the other tile's softmax runs;
+//               works on one tile while the other tile's softmax runs; each waits for V, K
+//               and P before its turn, so the turn is the last wait before its MMAs;
 //   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: one thread per query row
 //               (= TMEM lane). tcgen05.ld of the S row; masks (causal / q_offset / kv_lengths
 //               as one prefix bound per row, boolean mask bytes or partial-block bits); optional

@@ -210,28 +210,6 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 2^x for a pair on the FMA pipe, for x <= 8 (Cody-Waite style range reduction x = n + f with
-// n = round(x), f in [-1/2, 1/2], then 2^f by a degree-3 polynomial fitted for this library to
-// the minimum of the maximum relative error on that interval, 7.5e-5 = 2^-13.7 including the
-// float32 rounding of the scheme, and 2^n added to the exponent field). x is clamped at -125,
-// so inputs below it give ~2^-125 instead of 0: callers use it only where x is finite and
-// never far below the row maximum matters (rows whose logits are all finite).
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer in the low bits
-  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261096f, c3 = 0.05517150f;
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  float t0, t1, n0, n1, f0, f1, q0, q1;
-  add2(t0, t1, x0, x1, kMagic, kMagic);
-  add2(n0, n1, t0, t1, -kMagic, -kMagic);
-  add2(f0, f1, x0, x1, -n0, -n1);
-  fma2(q0, q1, c3, c3, f0, f1, c2, c2);
-  fma2(q0, q1, q0, q1, f0, f1, c1, c1);
-  fma2(q0, q1, q0, q1, f0, f1, c0, c0);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
 // max(a, b, c) in one instruction (three-input form of max.f32 on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
