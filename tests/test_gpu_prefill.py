@@ -115,6 +115,22 @@ def test_prefill_bias_layouts(D, layout, causal):
     assert_matches(out, want, 1e-2, f"bias {layout} D={D}")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_bias_with_block_info(D):
+    # a 16-bit bias (through shared-memory tiles at head_dim 64) together with the partial-block
+    # bits of a block-sparse mask
+    w = si.scaled(si.BLOCK_SPARSE, nheads=4, q_len=640, kv_len=768, block=128)
+    cls = si.block_classes(w)
+    mask = si.mask_device(w, cls, DEV)
+    info = sdpa.build_block_mask_info(mask, 128, 128)
+    rng = _rng(21 + D)
+    q, k, v = _qkv(22 + D, 1, 640, 768, 4, 4, D, torch.float16)
+    bias = torch.from_numpy(rng.standard_normal((4, 640, 768)).astype(np.float32)).to(torch.float16)
+    out = run(q, k, v, bias.to(DEV), block_info=info)
+    want = oracle.sdpa_forward(f64(q), f64(k), f64(v), bias=f64(bias), mask=mask.cpu().numpy()[None])
+    assert_matches(out, want, 1e-2, f"bias + block info D={D}")
+
+
 def test_prefill_block_info():
     w = si.scaled(si.BLOCK_SPARSE, nheads=4, q_len=600, kv_len=900, block=128)
     cls = si.block_classes(w)
