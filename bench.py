@@ -85,14 +85,20 @@ def profiled_traffic(summary, sources):
 
 # ---- distributed plumbing -------------------------------------------------------------------
 
-def init_dist(n_gpus):
+def init_dist(n_gpus, backend=None):
+    """Process group from the torchrun environment (one rank per GPU over NCCL; gloo when
+    there is no GPU, which the CPU tests use)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(backend, timeout=timeout)
     return rank, world, local
 
 
@@ -102,9 +108,11 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest x over the ranks (device times: the job takes as long as its slowest rank)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
