@@ -66,6 +66,10 @@ def load(path: str | None = None):
         lib = ctypes.CDLL(lib_path)
         lib.oracle_sdpa_forward.argtypes = [ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p]
         lib.oracle_sdpa_forward.restype = ctypes.c_int
+        lib.oracle_sdpa_forward_packed.argtypes = [
+            ctypes.POINTER(_Problem), ctypes.c_int64, _i64p, _i64p, ctypes.c_int64, _f64p, _f64p,
+            _f64p, _f64p]
+        lib.oracle_sdpa_forward_packed.restype = ctypes.c_int
         lib.oracle_cache_update_at_index.argtypes = [
             _f64p, _f64p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
             ctypes.c_int64, _i64p]
@@ -175,6 +179,58 @@ def sdpa_forward(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_o
                                  _ptr(v, _f64p), _ptr(out, _f64p))
     if rc != 0:
         raise OracleError(f"oracle_sdpa_forward failed with code {rc}")
+    return out
+
+
+def sdpa_forward_packed(q, k, v, q_segments, kv_segments=None, maxlen=None, scale=None,
+                        is_causal=False, q_offset=0, q_lengths=None, kv_lengths=None,
+                        kv_head_rule: str = "contiguous", lib=None) -> np.ndarray:
+    """scaled_dot_product_attention(query, key, value; q_segments, kv_segments, maxlen, scale,
+    is_causal, q_offset, q_lengths, kv_lengths) on packed sequences, in float64.
+
+    q: (total_q, H, dqk); k: (total_kv, Hkv, dqk); v: (total_kv, Hkv, dv), the sequences one
+    after the other with no batch axis; returns (total_q, H, dv). q_segments / kv_segments:
+    the lengths of the sequences (kv_segments defaults to q_segments); q_offset, q_lengths
+    and kv_lengths take one entry per sequence (or one integer for all).
+    """
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    Lq, H, D = q.shape
+    Lk, Hkv, Dk = k.shape
+    Dv = v.shape[2]
+    if v.shape[:2] != (Lk, Hkv) or Dk != D:
+        raise ValueError("inconsistent q/k/v shapes")
+    qs = np.ascontiguousarray(np.asarray(q_segments, dtype=np.int64).reshape(-1))
+    nseg = qs.shape[0]
+    ks = None if kv_segments is None else np.ascontiguousarray(
+        np.asarray(kv_segments, dtype=np.int64).reshape(-1))
+    if ks is not None and ks.shape != (nseg,):
+        raise ValueError("kv_segments must have one entry per query segment")
+    p = _Problem()
+    p.batch, p.q_len, p.kv_len, p.nheads, p.nkvheads, p.dqk, p.dv = 1, Lq, Lk, H, Hkv, D, Dv
+    p.scale = float("nan") if scale is None else float(scale)
+    p.causal = {False: 0, True: 1, "bottom_right": 2}[is_causal]
+    p.kv_head_rule = {"contiguous": 0, "interleaved": 1}[kv_head_rule]
+    keep = [qs] + ([ks] if ks is not None else [])
+    qo = np.asarray(q_offset, dtype=np.int64)
+    if qo.ndim == 0:
+        p.q_offset_scalar = int(qo)
+    else:
+        qo = _per_batch(qo, nseg)
+        keep.append(qo)
+        p.q_offset = _ptr(qo, _i64p)
+    for name, val in (("q_lengths", q_lengths), ("kv_lengths", kv_lengths)):
+        arr = _per_batch(val, nseg)
+        if arr is not None:
+            keep.append(arr)
+            setattr(p, name, _ptr(arr, _i64p))
+    out = np.zeros((Lq, H, Dv), dtype=np.float64)
+    rc = lib.oracle_sdpa_forward_packed(
+        ctypes.byref(p), nseg, _ptr(qs, _i64p), None if ks is None else _ptr(ks, _i64p),
+        -1 if maxlen is None else int(maxlen), _ptr(q, _f64p), _ptr(k, _f64p), _ptr(v, _f64p),
+        _ptr(out, _f64p))
+    if rc != 0:
+        raise OracleError(f"oracle_sdpa_forward_packed failed with code {rc}")
     return out
 
 

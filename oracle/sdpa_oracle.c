@@ -185,6 +185,49 @@ int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const dou
   return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
+/* Packed sequences (the entry's keywords q_segments, kv_segments, maxlen and its paragraph
+ * "Packed sequences"): query holds nseg sequences of q_segments[s] rows one after the other,
+ * key and value nseg sequences of kv_segments[s] rows; the s-th query segment attends to the
+ * s-th key/value segment only, exactly as batch element s of a padded batch would. Here p
+ * describes the packed arrays: batch = 1, q_len / kv_len the total lengths, and q_offset,
+ * q_lengths, kv_lengths (when given) hold one entry per segment. The segment lengths must add
+ * up to the total lengths, no length may be negative, and maxlen (when >= 0) must be at least
+ * every segment; a bias or a mask is an error. */
+int oracle_sdpa_forward_packed(const oracle_sdpa_problem* p, int64_t nseg,
+                               const int64_t* q_segments, const int64_t* kv_segments,
+                               int64_t maxlen, const double* q, const double* k,
+                               const double* v, double* out) {
+  int rc = check_problem(p);
+  if (rc) return rc;
+  if (p->batch != 1 || nseg < 0 || (nseg > 0 && !q_segments)) return ORACLE_ERR_ARG;
+  if (p->bias || p->mask) return ORACLE_ERR_ARG;
+  const int64_t* kvs = kv_segments ? kv_segments : q_segments; /* kv_segments defaults */
+  int64_t q_tot = 0, kv_tot = 0;
+  for (int64_t s = 0; s < nseg; ++s) {
+    if (q_segments[s] < 0 || kvs[s] < 0) return ORACLE_ERR_ARG;
+    if (maxlen >= 0 && (q_segments[s] > maxlen || kvs[s] > maxlen)) return ORACLE_ERR_RANGE;
+    q_tot += q_segments[s];
+    kv_tot += kvs[s];
+  }
+  if (q_tot != p->q_len || kv_tot != p->kv_len) return ORACLE_ERR_ARG;
+  const int64_t H = p->nheads, Hkv = p->nkvheads;
+  int64_t q0 = 0, k0 = 0;
+  for (int64_t s = 0; s < nseg; ++s) {
+    oracle_sdpa_problem ps = *p;
+    ps.q_len = q_segments[s];
+    ps.kv_len = kvs[s];
+    ps.q_offset = p->q_offset ? p->q_offset + s : NULL;
+    ps.q_lengths = p->q_lengths ? p->q_lengths + s : NULL;
+    ps.kv_lengths = p->kv_lengths ? p->kv_lengths + s : NULL;
+    rc = oracle_sdpa_forward(&ps, q + q0 * H * p->dqk, k + k0 * Hkv * p->dqk,
+                             v + k0 * Hkv * p->dv, out + q0 * H * p->dv);
+    if (rc) return rc;
+    q0 += q_segments[s];
+    k0 += kvs[s];
+  }
+  return ORACLE_OK;
+}
+
 /* Writing new keys/values into a KV cache at a per-sequence position (the Keras issue
  * "MultiHeadAttention is missing a position_bias call argument": `cache_update_index`; the
  * Flax discussion's cached_key/cached_value, shaped (batch, len, heads, head_dim)):

@@ -382,6 +382,134 @@ def printed_example_shapes(lib):
         assert np.isfinite(out).all()
 
 
+# ---- packed sequences (keywords q_segments, kv_segments, maxlen; paragraph "Packed sequences")
+
+def _brute_packed(q, k, v, qs, ks, causal=False, q_offset=None, q_lengths=None, kv_lengths=None):
+    """Pure-Python packed attention on tiny inputs: every (segment, query row, head) with
+    math.exp over its own segment's keys; kv head h // (H/Hkv)."""
+    Lq, H, D = q.shape
+    Hkv, Dv = k.shape[1], v.shape[2]
+    out = np.zeros((Lq, H, Dv))
+    q0 = k0 = 0
+    for s in range(len(qs)):
+        ql = qs[s] if q_lengths is None else q_lengths[s]
+        kl = ks[s] if kv_lengths is None else kv_lengths[s]
+        off = 0 if q_offset is None else q_offset[s]
+        if causal == "bottom_right":
+            off = kl - ql
+        for i in range(qs[s]):
+            for h in range(H):
+                if i >= ql:
+                    continue
+                g = h // (H // Hkv)
+                keys = [j for j in range(ks[s]) if j < kl and (not causal or j <= off + i)]
+                if not keys:
+                    out[q0 + i, h] = float("nan")
+                    continue
+                x = [sum(q[q0 + i, h, c] * k[k0 + j, g, c] for c in range(D)) / math.sqrt(D) for j in keys]
+                m = max(x)
+                w = [math.exp(t - m) for t in x]
+                z = sum(w)
+                for e in range(Dv):
+                    out[q0 + i, h, e] = sum(w[n] * v[k0 + j, g, e] for n, j in enumerate(keys)) / z
+        q0 += qs[s]
+        k0 += ks[s]
+    return out
+
+
+@pin
+def packed_brute_force(lib):
+    """Each query segment attends its own key/value segment only, as a batch element of a
+    padded batch would, with is_causal, q_offset, q_lengths and kv_lengths taken per segment;
+    checked against pure-Python loops (GQA, unequal q/kv segments, an empty segment, a
+    query row with no key, head dims 3 and 2)."""
+    rng = _rng(61)
+    qs, ks = [3, 0, 4, 2], [2, 3, 5, 1]
+    q = rng.standard_normal((sum(qs), 4, 3))
+    k = rng.standard_normal((sum(ks), 2, 3))
+    v = rng.standard_normal((sum(ks), 2, 2))
+    for kw in (dict(), dict(causal=True, q_offset=[0, 1, 1, -1]),
+               dict(causal=True, q_offset=[1, 0, 2, 0], q_lengths=[2, 0, 4, 1], kv_lengths=[2, 1, 4, 1]),
+               dict(causal="bottom_right", q_lengths=[3, 0, 3, 2], kv_lengths=[2, 3, 4, 1])):
+        want = _brute_packed(q, k, v, qs, ks, **kw)
+        got = oracle.sdpa_forward_packed(q, k, v, qs, ks, is_causal=kw.get("causal", False),
+                                         q_offset=kw.get("q_offset", 0), q_lengths=kw.get("q_lengths"),
+                                         kv_lengths=kw.get("kv_lengths"), lib=lib)
+        assert (np.isnan(got) == np.isnan(want)).all()
+        _close(np.nan_to_num(got), np.nan_to_num(want))
+
+
+@pin
+def packed_first_query_of_each_causal_segment(lib):
+    """With is_causal and q_offset 0, the first query of a segment sees only the segment's
+    first key, so its output is that key's value (kv_segments defaulting to q_segments)."""
+    rng = _rng(62)
+    segs = [5, 12, 3, 1, 7]
+    x = rng.standard_normal((sum(segs), 2, 6))
+    y = oracle.sdpa_forward_packed(x, x, x, segs, is_causal=True, lib=lib)
+    start = np.cumsum([0] + segs[:-1])
+    _close(y[start], x[start], 1e-15)
+
+
+@pin
+def packed_segments_are_isolated(lib):
+    """Changing the keys and values of one segment changes that segment's output only."""
+    rng = _rng(63)
+    qs, ks = [6, 9, 4], [7, 5, 8]
+    q = rng.standard_normal((sum(qs), 4, 8))
+    k = rng.standard_normal((sum(ks), 2, 8))
+    v = rng.standard_normal((sum(ks), 2, 8))
+    a = oracle.sdpa_forward_packed(q, k, v, qs, ks, lib=lib)
+    k2, v2 = k.copy(), v.copy()
+    k2[7:12] = rng.standard_normal((5, 2, 8))
+    v2[7:12] = rng.standard_normal((5, 2, 8))
+    b = oracle.sdpa_forward_packed(q, k2, v2, qs, ks, lib=lib)
+    _close(a[:6], b[:6], 0.0)
+    _close(a[15:], b[15:], 0.0)
+    assert np.abs(a[6:15] - b[6:15]).min() > 0
+
+
+@pin
+def packed_equals_torch_per_segment(lib):
+    """Segment by segment, packed attention is PyTorch's float64 routine on that segment
+    alone (GQA by repeated heads, causal with per-segment q_offset as a boolean mask)."""
+    rng = _rng(64)
+    qs, ks, off = [33, 17, 64], [40, 17, 70], [7, 0, 6]
+    q = rng.standard_normal((sum(qs), 6, 16))
+    k = rng.standard_normal((sum(ks), 2, 16))
+    v = rng.standard_normal((sum(ks), 2, 12))
+    got = oracle.sdpa_forward_packed(q, k, v, qs, ks, is_causal=True, q_offset=off, lib=lib)
+    q0 = k0 = 0
+    for s in range(3):
+        qq = q[None, q0:q0 + qs[s]]
+        kk = np.repeat(k[None, k0:k0 + ks[s]], 3, axis=2)
+        vv = np.repeat(v[None, k0:k0 + ks[s]], 3, axis=2)
+        i = np.arange(qs[s])[:, None]
+        j = np.arange(ks[s])[None, :]
+        want = _torch_sdpa(qq, kk, vv, attn_mask=(j <= off[s] + i))
+        _close(got[q0:q0 + qs[s]], want[0])
+        q0 += qs[s]
+        k0 += ks[s]
+
+
+@pin
+def packed_printed_example_and_errors(lib):
+    """Examples: x of size (16, 8, 20) with q_segments [5, 12, 3] and is_causal keeps its size.
+    The segment lengths must add up to the array lengths, and maxlen must be at least every
+    segment."""
+    ex = json.load(open(os.path.join(GOLDEN, "printed_examples.json")))["examples"][4]
+    x = _rng(65).random(tuple(reversed(ex["query"])))
+    y = oracle.sdpa_forward_packed(x, x, x, ex["q_segments"], is_causal=ex["is_causal"], maxlen=12, lib=lib)
+    assert y.shape == tuple(reversed(ex["output"])) and np.isfinite(y).all()
+    for bad in (dict(q_segments=[5, 12, 2]), dict(q_segments=[5, 12, 3], maxlen=11),
+                dict(q_segments=[5, 12, 3], kv_segments=[5, 13, 3]), dict(q_segments=[6, -1, 15])):
+        try:
+            oracle.sdpa_forward_packed(x, x, x, lib=lib, **bad)
+        except oracle.OracleError:
+            continue
+        raise AssertionError(f"accepted {bad}")
+
+
 # ---- cache update and decode ----------------------------------------------------------------
 
 @pin

@@ -34,6 +34,13 @@ MUTANTS = {
     "block_class_swapped": ("(set == cells ? 2 : 1)", "(set == cells ? 1 : 2)"),
     "block_bits_reversed": ("word |= (1u << c);", "word |= (1u << (31 - c));"),
     "block_full_at_edge": ("(set == cells ? 2 : 1)", "(set == bq * bk ? 2 : 1)"),
+    # packed mutants move starts only toward lower addresses, so every access stays in bounds
+    "packed_kv_segments_ignored": ("kv_segments ? kv_segments : q_segments;", "q_segments;"),
+    "packed_query_start": ("q + q0 * H * p->dqk", "q + q0 * Hkv * p->dqk"),
+    "packed_key_start": ("k + k0 * Hkv * p->dqk", "k + k0 * p->dqk"),
+    "packed_out_start": ("out + q0 * H * p->dv", "out + q0 * Hkv * p->dv"),
+    "packed_first_offset_only": ("p->q_offset ? p->q_offset + s", "p->q_offset ? p->q_offset"),
+    "packed_kv_lengths_first_only": ("p->kv_lengths ? p->kv_lengths + s", "p->kv_lengths ? p->kv_lengths"),
 }
 
 
