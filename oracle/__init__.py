@@ -66,6 +66,9 @@ def load(path: str | None = None):
         lib = ctypes.CDLL(lib_path)
         lib.oracle_sdpa_forward.argtypes = [ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p]
         lib.oracle_sdpa_forward.restype = ctypes.c_int
+        lib.oracle_sdpa_backward.argtypes = [
+            ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p]
+        lib.oracle_sdpa_backward.restype = ctypes.c_int
         lib.oracle_sdpa_forward_packed.argtypes = [
             ctypes.POINTER(_Problem), ctypes.c_int64, _i64p, _i64p, ctypes.c_int64, _f64p, _f64p,
             _f64p, _f64p]
@@ -180,6 +183,53 @@ def sdpa_forward(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_o
     if rc != 0:
         raise OracleError(f"oracle_sdpa_forward failed with code {rc}")
     return out
+
+
+def sdpa_backward(q, k, v, dout, mask=None, scale=None, is_causal=False, q_offset=0,
+                  q_lengths=None, kv_lengths=None, lib=None):
+    """Gradient of the fused implementation for the loss sum(dout * out): returns
+    (dq, dk, dv, dscale) in float64, with the shapes of q, k, v and a float. Rows with no
+    attended key and rows past q_lengths take no part. No bias (a call with a bias takes the
+    materialized implementation under automatic differentiation)."""
+    lib = lib or load()
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Lq, H, D = q.shape
+    Bk, Lk, Hkv, Dk = k.shape
+    Dv = v.shape[3]
+    if Bk != B or v.shape[:3] != (B, Lk, Hkv) or Dk != D or dout.shape != (B, Lq, H, Dv):
+        raise ValueError("inconsistent q/k/v/dout shapes")
+    p = _Problem()
+    p.batch, p.q_len, p.kv_len, p.nheads, p.nkvheads, p.dqk, p.dv = B, Lq, Lk, H, Hkv, D, Dv
+    p.scale = float("nan") if scale is None else float(scale)
+    p.causal = {False: 0, True: 1, "bottom_right": 2}[is_causal]
+    keep = []
+    qo = np.asarray(q_offset, dtype=np.int64)
+    if qo.ndim == 0:
+        p.q_offset_scalar = int(qo)
+    else:
+        qo = _per_batch(qo, B)
+        keep.append(qo)
+        p.q_offset = _ptr(qo, _i64p)
+    for name, val in (("q_lengths", q_lengths), ("kv_lengths", kv_lengths)):
+        arr = _per_batch(val, B)
+        if arr is not None:
+            keep.append(arr)
+            setattr(p, name, _ptr(arr, _i64p))
+    if mask is not None:
+        base, st = _broadcast4(np.asarray(mask).astype(np.uint8), np.uint8, B, H, Lq, Lk)
+        keep.append(base)
+        p.mask = _ptr(base, _u8p)
+        p.mask_stride = (ctypes.c_int64 * 4)(*st)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    ds = np.zeros(1, dtype=np.float64)
+    rc = lib.oracle_sdpa_backward(ctypes.byref(p), _ptr(q, _f64p), _ptr(k, _f64p), _ptr(v, _f64p),
+                                  _ptr(dout, _f64p), _ptr(dq, _f64p), _ptr(dk, _f64p), _ptr(dv, _f64p),
+                                  _ptr(ds, _f64p))
+    if rc != 0:
+        raise OracleError(f"oracle_sdpa_backward failed with code {rc}")
+    return dq, dk, dv, float(ds[0])
 
 
 def sdpa_forward_packed(q, k, v, q_segments, kv_segments=None, maxlen=None, scale=None,

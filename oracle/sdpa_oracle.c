@@ -185,6 +185,119 @@ int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const dou
   return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
+/* The gradient of the fused implementation (paragraph "Fused implementation": the fused
+ * implementation has a gradient with respect to query, key, value and scale, and a query that
+ * attends to no key, whose output is NaN, takes no part in it). For the loss
+ * L = sum over output elements of dout * out, with w_j the softmax weights of a row and
+ * x_j = scale * q.k_j its attended logits:
+ *   dv_j    += w_j * dout_i
+ *   dw_j     = dout_i . v_j
+ *   dx_j     = w_j * (dw_j - sum_l w_l dw_l)
+ *   dq_i     = scale * sum_j dx_j k_j
+ *   dk_j    += scale * dx_j q_i
+ *   dscale  += sum_j dx_j (q_i . k_j)
+ * summed over the query heads that share a key/value head. Rows past q_lengths (constant zero)
+ * and rows with no attended key contribute nothing and get dq = 0. A bias is an error: under
+ * automatic differentiation a call with a bias takes the materialized implementation. */
+int oracle_sdpa_backward(const oracle_sdpa_problem* p, const double* q, const double* k,
+                         const double* v, const double* dout, double* dq, double* dk, double* dv,
+                         double* dscale) {
+  int rc = check_problem(p);
+  if (rc) return rc;
+  if (p->bias || p->kv_head_rule != 0) return ORACLE_ERR_ARG;
+  const int64_t B = p->batch, Lq = p->q_len, Lk = p->kv_len, H = p->nheads, Hkv = p->nkvheads;
+  const int64_t D = p->dqk, Dv = p->dv, group = H / Hkv;
+  const double scale = isnan(p->scale) ? 1.0 / sqrt((double)D) : p->scale;
+  memset(dq, 0, sizeof(double) * (size_t)(B * Lq * H * D));
+  memset(dk, 0, sizeof(double) * (size_t)(B * Lk * Hkv * D));
+  memset(dv, 0, sizeof(double) * (size_t)(B * Lk * Hkv * Dv));
+  double total = 0.0;
+  int failed = 0;
+  /* each (batch, key/value head) owns its rows of dk and dv */
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : total)
+  for (int64_t bg = 0; bg < B * Hkv; ++bg) {
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    double* x = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+    double* dw = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+    unsigned char* ok = (unsigned char*)malloc((size_t)(Lk > 0 ? Lk : 1));
+    if (!x || !dw || !ok) {
+#pragma omp atomic write
+      failed = 1;
+      free(x);
+      free(dw);
+      free(ok);
+      continue;
+    }
+    const int64_t qlen_b = p->q_lengths ? p->q_lengths[b] : Lq;
+    const int64_t kvlen_b = p->kv_lengths ? p->kv_lengths[b] : Lk;
+    int64_t off = 0;
+    if (p->causal == 1) off = p->q_offset ? p->q_offset[b] : p->q_offset_scalar;
+    if (p->causal == 2) off = kvlen_b - qlen_b;
+    for (int64_t h = g * group; h < (g + 1) * group; ++h) {
+      for (int64_t i = 0; i < qlen_b && i < Lq; ++i) {
+        const double* qi = q + ((b * Lq + i) * H + h) * D;
+        const double* doi = dout + ((b * Lq + i) * H + h) * Dv;
+        double m = -INFINITY;
+        int64_t n = 0;
+        for (int64_t j = 0; j < Lk; ++j) {
+          int a = (j < kvlen_b);
+          if (p->causal != 0 && !(j <= off + i)) a = 0;
+          if (p->mask && !p->mask[j * p->mask_stride[0] + i * p->mask_stride[1] +
+                                  h * p->mask_stride[2] + b * p->mask_stride[3]])
+            a = 0;
+          ok[j] = (unsigned char)a;
+          if (!a) continue;
+          const double* kj = k + ((b * Lk + j) * Hkv + g) * D;
+          double dot = 0.0;
+          for (int64_t c = 0; c < D; ++c) dot += qi[c] * kj[c];
+          x[j] = scale * dot;
+          if (x[j] > m) m = x[j];
+          ++n;
+        }
+        if (n == 0) continue; /* NaN row: no part in the gradient */
+        double z = 0.0;
+        for (int64_t j = 0; j < Lk; ++j)
+          if (ok[j]) {
+            x[j] = exp(x[j] - m);
+            z += x[j];
+          }
+        double wdw = 0.0;
+        for (int64_t j = 0; j < Lk; ++j) {
+          if (!ok[j]) continue;
+          x[j] /= z; /* now the weight w_j */
+          const double* vj = v + ((b * Lk + j) * Hkv + g) * Dv;
+          double t = 0.0;
+          for (int64_t e = 0; e < Dv; ++e) t += doi[e] * vj[e];
+          dw[j] = t;
+          wdw += x[j] * t;
+        }
+        double* dqi = dq + ((b * Lq + i) * H + h) * D;
+        for (int64_t j = 0; j < Lk; ++j) {
+          if (!ok[j]) continue;
+          const double dx = x[j] * (dw[j] - wdw);
+          const double* kj = k + ((b * Lk + j) * Hkv + g) * D;
+          double* dkj = dk + ((b * Lk + j) * Hkv + g) * D;
+          double* dvj = dv + ((b * Lk + j) * Hkv + g) * Dv;
+          double dot = 0.0;
+          for (int64_t c = 0; c < D; ++c) {
+            dot += qi[c] * kj[c];
+            dqi[c] += scale * dx * kj[c];
+            dkj[c] += scale * dx * qi[c];
+          }
+          for (int64_t e = 0; e < Dv; ++e) dvj[e] += x[j] * doi[e];
+          total += dx * dot;
+        }
+      }
+    }
+    free(x);
+    free(dw);
+    free(ok);
+  }
+  if (failed) return ORACLE_ERR_NOMEM;
+  if (dscale) *dscale = total;
+  return ORACLE_OK;
+}
+
 /* Packed sequences (the entry's keywords q_segments, kv_segments, maxlen and its paragraph
  * "Packed sequences"): query holds nseg sequences of q_segments[s] rows one after the other,
  * key and value nseg sequences of kv_segments[s] rows; the s-th query segment attends to the

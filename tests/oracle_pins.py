@@ -382,6 +382,115 @@ def printed_example_shapes(lib):
         assert np.isfinite(out).all()
 
 
+# ---- the fused gradient (paragraph "Fused implementation") -----------------------------------
+
+def _loss(q, k, v, dout, lib, **kw):
+    """sum(dout * out) over the rows that attend some key (NaN rows take no part)."""
+    out = oracle.sdpa_forward(q, k, v, lib=lib, **kw)
+    return float(np.nansum(dout * out))
+
+
+def _central(f, x, h=1e-6):
+    """Central differences of the scalar f with respect to every element of x (in place)."""
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        idx = it.multi_index
+        old = x[idx]
+        x[idx] = old + h
+        up = f()
+        x[idx] = old - h
+        down = f()
+        x[idx] = old
+        g[idx] = (up - down) / (2 * h)
+    return g
+
+
+@pin
+def backward_finite_differences(lib):
+    """dq, dk, dv and dscale are the derivatives of sum(dout * out): checked element by element
+    against central differences of the (separately pinned) forward, with GQA, dv != dqk,
+    causal offsets, kv_lengths, q_lengths, a mask and a row that attends no key."""
+    rng = _rng(71)
+    q, k, v = _qkv(rng, 2, 4, 5, 4, 2, 3, 2)
+    dout = rng.standard_normal((2, 4, 4, 2))
+    mask = rng.random((1, 4, 4, 5)) < 0.7
+    cases = (dict(is_causal=True, q_offset=[1, -1], kv_lengths=[5, 3], scale=0.7),
+             dict(mask=mask, q_lengths=[3, 4], kv_lengths=[4, 5]),
+             dict(is_causal="bottom_right", q_lengths=[2, 4], kv_lengths=[4, 2]))
+    for kw in cases:
+        dq, dk, dv, ds = oracle.sdpa_backward(q, k, v, dout, lib=lib, **kw)
+        f = lambda: _loss(q, k, v, dout, lib, **kw)
+        _close(dq, _central(f, q), 1e-6)
+        _close(dk, _central(f, k), 1e-6)
+        _close(dv, _central(f, v), 1e-6)
+        s0 = kw.get("scale", 1 / math.sqrt(3))
+        g = lambda s: _loss(q, k, v, dout, lib, **{**kw, "scale": s})
+        _close(ds, (g(s0 + 1e-6) - g(s0 - 1e-6)) / 2e-6, 1e-6)
+
+
+@pin
+def backward_equals_torch_autograd(lib):
+    """PyTorch's float64 autograd of its scaled_dot_product_attention (GQA by repeating each
+    key/value head over its group of query heads, which autograd sums back; causal; a
+    boolean mask)."""
+    rng = _rng(72)
+    q, k, v = _qkv(rng, 2, 9, 9, 6, 2, 8, 5)
+    dout = rng.standard_normal((2, 9, 6, 5))
+    mask = rng.random((2, 6, 9, 9)) < 0.8
+    mask[..., 0] = True  # every row keeps a key
+    for kw, tkw in ((dict(is_causal=True), dict(is_causal=True)),
+                    (dict(mask=mask), dict(attn_mask=torch.from_numpy(mask)))):
+        tq, tk, tv = (torch.from_numpy(a.copy()).requires_grad_(True) for a in (q, k, v))
+        kk = tk.repeat_interleave(3, dim=2).permute(0, 2, 1, 3)
+        vv = tv.repeat_interleave(3, dim=2).permute(0, 2, 1, 3)
+        out = torch.nn.functional.scaled_dot_product_attention(tq.permute(0, 2, 1, 3), kk, vv, **tkw)
+        out.permute(0, 2, 1, 3).backward(torch.from_numpy(dout))
+        dq, dk, dv, _ = oracle.sdpa_backward(q, k, v, dout, lib=lib, **kw)
+        _close(dq, tq.grad.numpy())
+        _close(dk, tk.grad.numpy())
+        _close(dv, tv.grad.numpy())
+
+
+@pin
+def backward_invariants(lib):
+    """The weights of a row sum to one, so its logit gradients sum to zero: the key gradients
+    of a (batch, kv head) sum to zero, the value gradients sum to the dout of the rows that
+    attend some key, and scale * dscale = sum of q . dq."""
+    rng = _rng(73)
+    q, k, v = _qkv(rng, 2, 6, 7, 4, 2, 5, 3)
+    dout = rng.standard_normal((2, 6, 4, 3))
+    kw = dict(is_causal=True, q_offset=[0, -2], scale=0.45)
+    dq, dk, dv, ds = oracle.sdpa_backward(q, k, v, dout, lib=lib, **kw)
+    _close(dk.sum(axis=1), np.zeros((2, 2, 5)))
+    rows = np.ones((2, 6), dtype=bool)
+    rows[1, :2] = False  # offset -2: the first two rows of batch 1 attend no key
+    want = np.stack([np.stack([dout[b][rows[b]][:, 2 * g:2 * g + 2].sum(axis=(0, 1)) for g in range(2)])
+                     for b in range(2)])
+    _close(dv.sum(axis=1), want)
+    _close(0.45 * ds, float((q * dq).sum()))
+
+
+@pin
+def backward_excludes_empty_and_padding_rows(lib):
+    """A row with no attended key (NaN output) and a row past q_lengths (zero output) take no
+    part: their dq is zero and their dout changes nothing."""
+    rng = _rng(74)
+    q, k, v = _qkv(rng, 2, 5, 6, 2, 2, 4)
+    dout = rng.standard_normal((2, 5, 2, 4))
+    kw = dict(q_lengths=[3, 5], kv_lengths=[6, 0])
+    a = oracle.sdpa_backward(q, k, v, dout, lib=lib, **kw)
+    _close(a[0][0, 3:], np.zeros((2, 2, 4)), 0.0)
+    _close(a[0][1], np.zeros((5, 2, 4)), 0.0)
+    d2 = dout.copy()
+    d2[0, 3:] = 100.0
+    d2[1] = -7.0
+    b = oracle.sdpa_backward(q, k, v, d2, lib=lib, **kw)
+    for x, y in zip(a[:3], b[:3]):
+        _close(x, y, 0.0)
+    assert a[3] == b[3]
+
+
 # ---- packed sequences (keywords q_segments, kv_segments, maxlen; paragraph "Packed sequences")
 
 def _brute_packed(q, k, v, qs, ks, causal=False, q_offset=None, q_lengths=None, kv_lengths=None):

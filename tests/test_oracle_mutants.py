@@ -34,6 +34,11 @@ MUTANTS = {
     "block_class_swapped": ("(set == cells ? 2 : 1)", "(set == cells ? 1 : 2)"),
     "block_bits_reversed": ("word |= (1u << c);", "word |= (1u << (31 - c));"),
     "block_full_at_edge": ("(set == cells ? 2 : 1)", "(set == bq * bk ? 2 : 1)"),
+    "backward_delta_sign": ("x[j] * (dw[j] - wdw)", "x[j] * (dw[j] + wdw)"),
+    "backward_dk_unscaled": ("dkj[c] += scale * dx * qi[c];", "dkj[c] += dx * qi[c];"),
+    "backward_dv_from_dx": ("dvj[e] += x[j] * doi[e];", "dvj[e] += dx * doi[e];"),
+    "backward_dscale_scaled": ("total += dx * dot;", "total += dx * dot * scale;"),
+    "backward_causal_off_by_one": ("!(j <= off + i)) a = 0;", "!(j < off + i)) a = 0;"),
     # packed mutants move starts only toward lower addresses, so every access stays in bounds
     "packed_kv_segments_ignored": ("kv_segments ? kv_segments : q_segments;", "q_segments;"),
     "packed_query_start": ("q + q0 * H * p->dqk", "q + q0 * Hkv * p->dqk"),
