@@ -295,6 +295,10 @@ def other_workloads(args, dev, world, ws, peaks):
         res["alibi_t5_bias"] = bias_workload(args, dev, world, ws)
     if "block_sparse" in args.workloads:
         res["block_sparse_mask"] = block_sparse_workload(args, dev, world, ws, peaks)
+    if "packed" in args.workloads:
+        res["packed_docs"] = packed_workload(args, dev, world, ws, peaks)
+    if "backward" in args.workloads:
+        res["fused_gradient"] = backward_workload(args, dev, world, ws, peaks)
     return res
 
 
@@ -370,6 +374,50 @@ def block_sparse_workload(args, dev, world, ws, peaks):
         "classification": {"ms": round(ms_c, 4), "GB/s": round(mask.numel() / (ms_c * 1e-3) / 1e9, 1),
                            "frac_hbm": round(mask.numel() / (ms_c * 1e-3) / 1e9 / peaks["hbm"], 4)},
         "kernel": sdpa.last_kernel()}
+
+
+def packed_workload(args, dev, world, ws, peaks):
+    """Packed sequences: documents of 64 to 4096 positions one after the other, each attending
+    causally to itself only (the segment scan and the attention kernel, every step)."""
+    import head_scaled_dot_sdpa_b200 as sdpa
+
+    w = si.PACKED_DOCS
+    segs = si.packed_segments(w)
+    q, k, v = [t.to(dev) for t in si.packed_qkv(w)]
+    seg = torch.tensor(segs, dtype=torch.int32, device=dev)
+    maxlen = max(segs)
+    out = torch.empty_like(q)
+    flops = 4.0 * w.head_dim * w.nheads * sum(causal_pairs(n, n) for n in segs)
+    step = lambda: sdpa.sdpa_forward_packed(q, k, v, seg, maxlen=maxlen, is_causal=True, out=out, workspace=ws)
+    per = time_steps(step, args.steps, args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "segments": len(segs), "maxlen": maxlen, "value": round(tf * world, 2),
+            "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16"], 4)},
+            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 2}
+
+
+def backward_workload(args, dev, world, ws, peaks):
+    """The fused gradient (dq, dk, dv, dscale) of the causal GQA prefill workload: 10*head_dim
+    flops per attended pair (the logits recomputed, dout.v, and the dv, dq and dk products)."""
+    import head_scaled_dot_sdpa_b200 as sdpa
+
+    w = si.CAUSAL_GQA_PREFILL
+    q, k, v = [t.to(dev) for t in si.qkv(w)]
+    dout = si.normal(si.rng_for(w.seed + 7), tuple(q.shape), w.dtype).to(dev)
+    out = sdpa.sdpa_forward(q, k, v, is_causal=True, workspace=ws)
+    flops = 10.0 * w.head_dim * w.batch * w.nheads * causal_pairs(w.q_len, w.kv_len)
+    step = lambda: sdpa.sdpa_backward(q, k, v, out, dout, is_causal=True, workspace=ws)
+    per = time_steps(step, max(3, args.steps // 4), args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name + "_backward", "value": round(tf * world, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16"], 5)},
+            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 3}
 
 
 # ---- CPU oracle ---------------------------------------------------------------------------------
@@ -452,7 +500,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--reference-heads", type=int, default=16)
-    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse",
+    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse,packed,backward",
                     help="comma list; without 'prefill' only the other workloads run (a profiling aid)")
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide the decode batch and the block-sparse length by this (small ncu cases)")

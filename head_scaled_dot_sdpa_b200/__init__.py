@@ -64,12 +64,23 @@ class Params(ctypes.Structure):
                 ("block_info", ctypes.POINTER(BlockMaskInfoStruct)), ("flags", ctypes.c_uint32)]
 
 
+class PackedSegments(ctypes.Structure):
+    _fields_ = [("nseg", ctypes.c_int32), ("maxlen", ctypes.c_int32), ("q_segments", ctypes.c_void_p),
+                ("kv_segments", ctypes.c_void_p)]
+
+
 _vp, _sz, _i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
 _PP = ctypes.POINTER(Params)
 _lib.sdpa_workspace_size.argtypes = [_PP]
 _lib.sdpa_workspace_size.restype = _sz
 _lib.sdpa_workspace_init.argtypes = [_vp, _sz, _vp]
 _lib.sdpa_forward.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sdpa_packed_workspace_size.argtypes = [_PP, ctypes.POINTER(PackedSegments)]
+_lib.sdpa_packed_workspace_size.restype = _sz
+_lib.sdpa_forward_packed.argtypes = [_PP, ctypes.POINTER(PackedSegments), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sdpa_backward_workspace_size.argtypes = [_PP]
+_lib.sdpa_backward_workspace_size.restype = _sz
+_lib.sdpa_backward.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sdpa_decode_with_cache.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.cache_update_at_index.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32,
                                        _i32, _vp, _vp, _vp]
@@ -80,7 +91,8 @@ _lib.build_block_mask_info.argtypes = [_vp, ctypes.POINTER(ctypes.c_int64), _i32
 _lib.sdpa_read_device_status.argtypes = [_vp, _vp]
 _lib.sdpa_last_error.restype = ctypes.c_char_p
 _lib.sdpa_last_kernel.restype = ctypes.c_char_p
-for _f in ("sdpa_workspace_init", "sdpa_forward", "sdpa_decode_with_cache", "cache_update_at_index",
+for _f in ("sdpa_workspace_init", "sdpa_forward", "sdpa_forward_packed", "sdpa_backward", "sdpa_decode_with_cache",
+           "cache_update_at_index",
            "build_block_mask_info", "sdpa_read_device_status"):
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -260,6 +272,101 @@ def sdpa_forward(q, k, v, bias=None, *, mask=None, scale=None, is_causal=False, 
     return out
 
 
+def sdpa_backward(q, k, v, out, dout, *, mask=None, scale=None, is_causal=False, q_offset=0,
+                  q_lengths=None, kv_lengths=None, block_info=None, workspace=None, stream=None):
+    """The gradient of the fused implementation for the loss sum(dout * out), where `out` is
+    sdpa_forward(q, k, v; ...) with the same arguments: returns (dq, dk, dv, dscale), dscale a
+    0-d float32 device tensor. Rows with no attended key and rows past q_lengths take no part.
+    No bias (the page's automatic differentiation takes the materialized implementation then)."""
+    _check_qkv(q, k, v)
+    for n, t in (("out", out), ("dout", dout)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype or t.shape != q.shape[:3] + (v.shape[3],):
+            raise ValueError(f"{n} must be a contiguous CUDA tensor of the output's shape and dtype")
+    keep = []
+    p = _params(q, k, v, bias=None, mask=mask, scale=scale, is_causal=is_causal, q_offset=q_offset,
+                q_lengths=q_lengths, kv_lengths=kv_lengths, block_info=block_info, flags=0, keep=keep)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dscale = torch.zeros((), dtype=torch.float32, device=q.device)
+    need = _lib.sdpa_backward_workspace_size(ctypes.byref(p))
+    if need == 0:
+        raise SdpaError(SDPA_ERR_INVALID_ARG, _lib.sdpa_last_error().decode())
+    ws = _workspace(q.device, need, workspace)
+    _check(_lib.sdpa_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(dq),
+                              _ptr(dk), _ptr(dv), dscale.data_ptr(), ws.ptr, ws.nbytes, _stream(stream)))
+    return dq, dk, dv, dscale
+
+
+def _segments(x, device, name):
+    """Segment lengths -> (device int32 tensor, host list or None). A host sequence is copied to
+    the device; a device tensor stays there."""
+    if isinstance(x, torch.Tensor):
+        if x.dim() != 1:
+            raise ValueError(f"{name} must be a vector of lengths")
+        t = x.to(device=device, dtype=torch.int32).contiguous()
+        return t, (None if x.is_cuda else [int(a) for a in x.tolist()])
+    lens = [int(a) for a in x]
+    return torch.tensor(lens, dtype=torch.int32, device=device), lens
+
+
+def sdpa_forward_packed(q, k, v, q_segments, kv_segments=None, *, maxlen=None, scale=None,
+                        is_causal=False, q_offset=0, q_lengths=None, kv_lengths=None, out=None,
+                        workspace=None, generic=False, stream=None):
+    """scaled_dot_product_attention(q, k, v; q_segments, kv_segments, maxlen, scale, is_causal,
+    q_offset, q_lengths, kv_lengths) on packed sequences: q (total_q, H, dqk), k (total_kv, Hkv,
+    dqk) and v (total_kv, Hkv, dv) hold the sequences one after the other; out is (total_q, H,
+    dv). q_offset / q_lengths / kv_lengths take one entry per sequence. Without maxlen, lengths
+    given as a device tensor are copied to the host to find it (which waits for the device)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{n} must be a contiguous 3-d CUDA tensor (total_len, heads, d)")
+        if t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k and v must share dtype and device")
+    if v.shape[:2] != k.shape[:2] or k.shape[2] != q.shape[2]:
+        raise ValueError("inconsistent q/k/v shapes")
+    dev = q.device
+    qs, q_host = _segments(q_segments, dev, "q_segments")
+    keep = [qs]
+    ks, kv_host = None, q_host
+    if kv_segments is not None:
+        ks, kv_host = _segments(kv_segments, dev, "kv_segments")
+        if ks.shape != qs.shape:
+            raise ValueError("kv_segments must have one entry per query segment")
+        keep.append(ks)
+    nseg = qs.shape[0]
+    if maxlen is None:
+        if q_host is None:
+            q_host = [int(a) for a in qs.cpu().tolist()]
+        if ks is None:
+            kv_host = q_host
+        elif kv_host is None:
+            kv_host = [int(a) for a in ks.cpu().tolist()]
+        maxlen = max(q_host + kv_host, default=0)
+    p = _params(q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0), bias=None, mask=None, scale=scale,
+                is_causal=is_causal, q_offset=0, q_lengths=None, kv_lengths=None, block_info=None,
+                flags=SDPA_FLAG_GENERIC_KERNEL if generic else 0, keep=keep)
+    if isinstance(q_offset, int):
+        p.q_offset_scalar = q_offset
+    else:
+        t = _per_batch(q_offset, nseg, dev, "q_offset")
+        keep.append(t)
+        p.q_offset = t.data_ptr()
+    for name, val in (("q_lengths", q_lengths), ("kv_lengths", kv_lengths)):
+        t = _per_batch(val, nseg, dev, name)
+        if t is not None:
+            keep.append(t)
+            setattr(p, name, t.data_ptr())
+    seg = PackedSegments(nseg, int(maxlen), qs.data_ptr(), None if ks is None else ks.data_ptr())
+    if out is None:
+        out = torch.empty(q.shape[:2] + (v.shape[2],), dtype=q.dtype, device=dev)
+    need = _lib.sdpa_packed_workspace_size(ctypes.byref(p), ctypes.byref(seg))
+    if need == 0:
+        raise SdpaError(SDPA_ERR_INVALID_ARG, _lib.sdpa_last_error().decode())
+    ws = _workspace(dev, need, workspace)
+    _check(_lib.sdpa_forward_packed(ctypes.byref(p), ctypes.byref(seg), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(out), ws.ptr, ws.nbytes, _stream(stream)))
+    return out
+
+
 def sdpa_decode_with_cache(q, k_new, v_new, k_cache, v_cache, cache_index, *, scale=None,
                            out=None, workspace=None, generic=False, stream=None):
     """Writes k_new/v_new (B, n_new, Hkv, d) into the caches (B, capacity, Hkv, d) at
@@ -343,6 +450,6 @@ def build_block_mask_info(mask, bq: int = 128, bk: int = 128, *, stream=None) ->
     return info
 
 
-__all__ = ["sdpa_forward", "sdpa_decode_with_cache", "cache_update_at_index",
+__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
            "build_block_mask_info", "BlockMaskInfo", "Workspace", "read_device_status",
            "last_kernel", "SdpaError", "lib"]

@@ -28,15 +28,28 @@ __device__ __forceinline__ void report(int* status, int code) {
 
 // Lengths, offsets: the arguments q_lengths, kv_lengths, q_offset and is_causal of
 // NNlib.scaled_dot_product_attention. Out-of-range lengths are clamped and reported.
+// With packed sequences (keywords q_segments / kv_segments, paragraph "Packed sequences") the
+// b-th segment plays the part of batch element b, its lengths bounding q_lengths / kv_lengths.
 __device__ __forceinline__ BatchInfo resolve_batch(const Problem& P, int b) {
   BatchInfo bi;
   bi.skip = false;
-  int ql = P.Lq, kl = P.Lk;
+  int qseg = P.Lq, kseg = P.Lk;
+  if (P.q_start) {
+    bi.q0 = P.q_start[b];
+    bi.k0 = P.kv_start[b];
+    qseg = P.q_start[b + 1] - (int)bi.q0;
+    kseg = P.kv_start[b + 1] - (int)bi.k0;
+  } else {
+    bi.q0 = (long long)b * P.Lq;
+    bi.k0 = (long long)b * P.Lk;
+  }
+  bi.q_rows = qseg;
+  int ql = qseg, kl = kseg;
   if (P.q_lengths) {
     ql = P.q_lengths[b];
-    if (ql < 0 || ql > P.Lq) {
+    if (ql < 0 || ql > qseg) {
       report(P.status, SDPA_ERR_DEVICE_CHECK);
-      ql = ql < 0 ? 0 : P.Lq;
+      ql = ql < 0 ? 0 : qseg;
     }
   }
   if (P.cache_index) {
@@ -46,9 +59,9 @@ __device__ __forceinline__ BatchInfo resolve_batch(const Problem& P, int b) {
   } else if (P.kv_lengths) {
     kl = P.kv_lengths[b];
   }
-  if (kl < 0 || kl > P.Lk) {
+  if (kl < 0 || kl > kseg) {
     report(P.status, SDPA_ERR_DEVICE_CHECK);
-    kl = kl < 0 ? 0 : P.Lk;
+    kl = kl < 0 ? 0 : kseg;
   }
   bi.q_len = ql;
   bi.kv_len = kl;

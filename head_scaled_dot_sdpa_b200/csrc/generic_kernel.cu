@@ -43,14 +43,17 @@ generic_attention_kernel(Problem P, const T* __restrict__ q, const T* __restrict
   const int b = (int)(row / ((long long)P.H * P.Lq));
   const int D = P.D, Dv = P.Dv;
 
+  // row (b, i, h) of a padded batch, or row i of packed sequence b (whose rows start at bi.q0;
+  // rows past the sequence belong to the next one and are left alone)
+  const BatchInfo bi = resolve_batch(P, b);
+  if (bi.skip || i >= bi.q_rows) return;
+  const long long qi = (bi.q0 + i) * P.H + h;
   float* qs = q_smem + warp * D;
-  const T* qrow = q + row * D;
+  const T* qrow = q + qi * D;
   for (int c = lane; c < D; c += 32) qs[c] = to_f32(qrow[c]);
   __syncwarp();
 
-  T* orow = out + row * Dv;
-  const BatchInfo bi = resolve_batch(P, b);
-  if (bi.skip) return;
+  T* orow = out + qi * Dv;
   if (i >= bi.q_len) {  // argument q_lengths: padding rows are zero
     for (int e = lane; e < Dv; e += 32) orow[e] = from_f32<T>(0.f);
     return;
@@ -71,7 +74,7 @@ generic_attention_kernel(Problem P, const T* __restrict__ q, const T* __restrict
     const long long j = j0 + lane;
     float s = -INFINITY;
     if (j < jend && mask_allows(P, b, h, i, (int)j)) {
-      const T* kr = k + (((long long)b * P.Lk + j) * P.Hkv + g) * D;
+      const T* kr = k + ((bi.k0 + j) * P.Hkv + g) * D;
       float acc = 0.f;
       for (int c = 0; c < D; ++c) acc = fmaf(qs[c], to_f32(kr[c]), acc);
       s = acc * P.scale;
@@ -88,7 +91,7 @@ generic_attention_kernel(Problem P, const T* __restrict__ q, const T* __restrict
     for (int t = 0; t < n; ++t) {
       const float pt = __shfl_sync(0xffffffffu, p, t);
       if (pt == 0.f) continue;  // warp-uniform
-      const T* vr = v + (((long long)b * P.Lk + j0 + t) * P.Hkv + g) * Dv;
+      const T* vr = v + ((bi.k0 + j0 + t) * P.Hkv + g) * Dv;
 #pragma unroll
       for (int u = 0; u < kMaxDvPerLane; ++u) {
         const int e = lane + 32 * u;

@@ -36,6 +36,12 @@ struct Problem {
   const uint32_t* brow_list;
   const uint32_t* bbits;
   int bi_nheads, bi_nqb, bi_nkb, bi_bq, bi_bk;
+  // packed sequences (q_segments / kv_segments): B is the number of segments and Lq / Lk the
+  // longest segment (maxlen); q_start / kv_start hold the first row of each segment in the
+  // packed arrays, B + 1 entries, the last one the total row count. Null for a padded batch.
+  const int32_t* q_start;
+  const int32_t* kv_start;
+  int Lq_total, Lk_total;    // rows of the packed arrays
   int* status;               // device status word (never null when a kernel runs)
   unsigned long long wait_timeout_ns;  // bound on every mbarrier wait of the tcgen05 kernel
   int selftest_stall;                  // SDPA_FLAG_SELFTEST_STALL
@@ -47,6 +53,8 @@ struct BatchInfo {
   int kv_len;  // valid keys
   int offset;  // causal offset (query i attends keys j <= offset + i)
   bool skip;   // decode: the cache index is out of range, leave this sequence alone
+  int q_rows;  // rows of this sequence in the query / output arrays (rows past it are not written)
+  long long q0, k0;  // first row of this sequence in the (rows, heads, dim) view of q / out, k / v
 };
 
 // Records the message sdpa_last_error() returns on this host thread.
@@ -68,6 +76,18 @@ cudaError_t launch_block_classify(const uint8_t* mask, const long long ms[3], in
                                   int Lk, int bq, int bk, uint8_t* cls, int32_t* count,
                                   uint32_t* list, uint32_t* bits, int* status,
                                   cudaStream_t stream);
+// Packed sequences: writes the first row of each query and key/value segment (exclusive prefix
+// sums of the lengths, clamped to the array rows; n + 1 entries each). A negative length, one
+// above maxlen, or lengths that do not add up to the array rows set SDPA_ERR_DEVICE_CHECK.
+cudaError_t launch_segment_starts(const int32_t* q_segments, const int32_t* kv_segments, int n,
+                                  int maxlen, int q_total, int kv_total, int32_t* q_start,
+                                  int32_t* kv_start, int* status, cudaStream_t stream);
+// The fused gradient (dq, dk, dv, dscale): three SIMT kernels. `ws` holds the per-row
+// log-sum-exp and delta = dout . out (backward_workspace_bytes).
+size_t backward_workspace_bytes(const Problem& P);
+cudaError_t launch_backward(const Problem& P, const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, void* dq, void* dk, void* dv, float* dscale, void* ws,
+                            cudaStream_t stream);
 bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v,
                        const void* out);
 size_t prefill_workspace_bytes(const Problem& P);

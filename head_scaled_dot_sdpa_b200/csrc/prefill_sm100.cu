@@ -106,8 +106,11 @@ size_t prefill_workspace_bytes(const Problem&) { return 0; }
 cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const void* v, void* out, void*,
                            cudaStream_t stream, const char** msg) {
   prefill::TensorMaps maps{};
-  if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
-      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B)) {
+  // packed sequences: one batch of all rows, each sequence read from its own first row
+  const bool packed = P.q_start != nullptr;
+  const int q_rows = packed ? P.Lq_total : P.Lq, kv_rows = packed ? P.Lk_total : P.Lk, nb = packed ? 1 : P.B;
+  if (!make_map(&maps.q, q, P.dtype, P.D, P.H, q_rows, nb) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, kv_rows, nb) ||
+      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, kv_rows, nb)) {
     if (msg) *msg = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }

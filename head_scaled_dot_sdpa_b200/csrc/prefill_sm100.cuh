@@ -105,6 +105,9 @@ struct QTile {
 struct Unit {
   int b, kvh;
   int q_len, kv_len, offset;
+  int q_rows;       // rows of the sequence in q / out; rows past it are another sequence's
+  int tq, tk, tb;   // TMA coordinates: first query row, first key row, batch index
+  long long o0;     // first row of the sequence in out viewed as (rows, heads, head_dim)
   QTile t[2];
 };
 
@@ -176,6 +179,14 @@ __device__ __forceinline__ Unit make_unit(const Problem& P, int u) {
   w.q_len = bi.q_len;
   w.kv_len = bi.kv_len;
   w.offset = bi.offset;
+  w.q_rows = bi.q_rows;
+  w.o0 = bi.q0;
+  // a padded batch is a 4-d map indexed by batch; packed sequences are one batch of all rows,
+  // each sequence starting at its own row
+  const bool packed = P.q_start != nullptr;
+  w.tq = packed ? (int)bi.q0 : 0;
+  w.tk = packed ? (int)bi.k0 : 0;
+  w.tb = packed ? 0 : w.b;
   w.t[0] = make_qtile(P, bi, hA, qA, true);
   w.t[1] = make_qtile(P, bi, hB, qB, haveB);
   if (!haveB) w.t[1].i0 = kNone;  // marks "no tile B"
@@ -353,7 +364,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
 #pragma unroll
           for (int s = 0; s < 2; ++s)
             if (w.t[s].n > 0)
-              for (int r = 0; r < C::kRegions; ++r) tma_prefetch_l2_4d(&maps.q, r * 64, w.t[s].h, w.t[s].i0, w.b);
+              for (int r = 0; r < C::kRegions; ++r) tma_prefetch_l2_4d(&maps.q, r * 64, w.t[s].h, w.tq + w.t[s].i0, w.tb);
         }
         __syncwarp();
 #pragma unroll
@@ -364,7 +375,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
             for (int r = 0; r < C::kRegions; ++r)
               tma_load_4d(q_smem + s * C::kTileBytes + r * kRegionBytes, &maps.q, &q_full[s], r * 64,
-                          w.t[s].h, w.t[s].i0, w.b);
+                          w.t[s].h, w.tq + w.t[s].i0, w.tb);
           }
           ++qc[s];
         }
@@ -381,7 +392,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               mbar_arrive_expect_tx(&k_full[ks], C::kTileBytes);
               for (int r = 0; r < C::kRegions; ++r)
                 tma_load_4d(k_smem + ks * C::kTileBytes + r * kRegionBytes, &maps.k, &k_full[ks], r * 64,
-                            w.kvh, kb * kBlockN, w.b);
+                            w.kvh, w.tk + kb * kBlockN, w.tb);
             }
           }
           if (prev_kb >= 0) {
@@ -392,7 +403,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               mbar_arrive_expect_tx(&v_full[vs], C::kTileBytes);
               for (int r = 0; r < C::kRegions; ++r)
                 tma_load_4d(v_smem + vs * C::kTileBytes + r * kRegionBytes, &maps.v, &v_full[vs], r * 64,
-                            w.kvh, prev_kb * kBlockN, w.b);
+                            w.kvh, w.tk + prev_kb * kBlockN, w.tb);
             }
           }
           if constexpr (kBias == kBiasTile) {
@@ -606,10 +617,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         const QTile qt = s ? w.t[1] : w.t[0];
         if (qt.i0 == kNone) continue;  // the unit has no tile B
         const int i = qt.i0 + r;
-        T* orow = out + (((long long)w.b * P.Lq + i) * P.H + qt.h) * D;
+        T* orow = out + ((w.o0 + i) * P.H + qt.h) * D;
         if (qt.n == 0) {
           // no key tile: NaN rows (nothing attended) or zero rows (past q_lengths)
-          if (i < P.Lq) {
+          if (i < w.q_rows) {
             const float val = (i >= w.q_len) ? 0.f : __int_as_float(0x7fc00000);
             const uint32_t wv = std::is_same<T, __half>::value ? pack_f16x2(val, val) : pack_bf16x2(val, val);
 #pragma unroll
@@ -793,7 +804,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           uint32_t o[32];
           tmem_ld32(lane_addr + ocol + c * 32, o);
           tmem_wait_ld();
-          if (i < P.Lq) {
+          if (i < w.q_rows) {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint32_t wv[4];

@@ -183,6 +183,116 @@ sdpa_status sdpa_forward(const sdpa_params* p, const void* q, const void* k, con
   return SDPA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The packed call as a problem over nseg sequences of at most maxlen rows; the segment starts
+// go in the workspace after the status word.
+sdpa_status resolve_packed(const sdpa_params* p, const sdpa_packed_segments* seg, sdpa::Problem* P,
+                           size_t* need) {
+  sdpa_status st = resolve(p, P);
+  if (st != SDPA_OK) return st;
+  if (!seg) return fail(SDPA_ERR_INVALID_ARG, "segments are NULL");
+  if (p->batch != 1)
+    return fail(SDPA_ERR_INVALID_ARG, "packed sequences have no batch axis: batch must be 1, got %d", p->batch);
+  if (p->bias || p->mask || p->block_info)
+    return fail(SDPA_ERR_INVALID_ARG, "a bias or a mask is not supported with packed sequences");
+  if (seg->nseg < 0 || seg->maxlen < 0) return fail(SDPA_ERR_INVALID_ARG, "negative nseg or maxlen");
+  if (seg->nseg > 0 && !seg->q_segments) return fail(SDPA_ERR_INVALID_ARG, "q_segments is NULL");
+  if (seg->nseg == 0 && (p->q_len > 0 || p->kv_len > 0))
+    return fail(SDPA_ERR_INVALID_ARG, "no segments for %d query and %d key rows", p->q_len, p->kv_len);
+  P->Lq_total = p->q_len;
+  P->Lk_total = p->kv_len;
+  P->B = seg->nseg;
+  P->Lq = seg->maxlen;
+  P->Lk = seg->maxlen;
+  *need = kStatusBytes + round256(sdpa::prefill_workspace_bytes(*P)) +
+          round256(2 * sizeof(int32_t) * ((size_t)seg->nseg + 1));
+  return SDPA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sdpa_packed_workspace_size(const sdpa_params* p, const sdpa_packed_segments* seg) {
+  sdpa::Problem P;
+  size_t need = 0;
+  if (resolve_packed(p, seg, &P, &need) != SDPA_OK) return 0;
+  return need;
+}
+
+sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed_segments* seg,
+                                const void* q, const void* k, const void* v, void* out,
+                                void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  sdpa::Problem P;
+  size_t need = 0;
+  sdpa_status st = resolve_packed(p, seg, &P, &need);
+  if (st != SDPA_OK) return st;
+  st = check_workspace(ws, ws_bytes, need);
+  if (st != SDPA_OK) return st;
+  if (P.Lq_total == 0) return SDPA_OK;
+  if (!q || !out || (P.Lk_total > 0 && (!k || !v)))
+    return fail(SDPA_ERR_INVALID_ARG, "q, k, v and out must not be NULL");
+  P.status = static_cast<int*>(ws);
+  void* scratch = static_cast<char*>(ws) + kStatusBytes;
+  int32_t* starts = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) +
+                                               round256(sdpa::prefill_workspace_bytes(P)));
+  P.q_start = starts;
+  P.kv_start = starts + P.B + 1;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = sdpa::launch_segment_starts(seg->q_segments, seg->kv_segments ? seg->kv_segments : seg->q_segments,
+                                              P.B, seg->maxlen, P.Lq_total, P.Lk_total, starts, starts + P.B + 1,
+                                              P.status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "segment scan launch");
+  if (P.Lq == 0) return SDPA_OK;  // maxlen 0: every segment is empty (or flagged by the scan)
+  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && P.Lk_total > 0 && sdpa::prefill_supported(P, q, k, v, out)) {
+    const char* msg = nullptr;
+    e = sdpa::launch_prefill(P, q, k, v, out, scratch, s, &msg);
+    if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");
+    g_last_kernel = "prefill_tcgen05";
+    return SDPA_OK;
+  }
+  if (!generic_ok(P))
+    return fail(SDPA_ERR_UNSUPPORTED, "head sizes dqk=%d dv=%d exceed the SIMT kernel's limits (1024, 256)",
+                P.D, P.Dv);
+  e = sdpa::launch_generic(P, q, k, v, out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "generic attention launch");
+  g_last_kernel = "generic_simt";
+  return SDPA_OK;
+}
+
+size_t sdpa_backward_workspace_size(const sdpa_params* p) {
+  sdpa::Problem P;
+  if (resolve(p, &P) != SDPA_OK) return 0;
+  return kStatusBytes + round256(sdpa::backward_workspace_bytes(P));
+}
+
+sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, const void* v,
+                          const void* out, const void* dout, void* dq, void* dk, void* dv,
+                          float* dscale, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  sdpa::Problem P;
+  sdpa_status st = resolve(p, &P);
+  if (st != SDPA_OK) return st;
+  if (p->bias)
+    return fail(SDPA_ERR_INVALID_ARG,
+                "the fused gradient takes no bias (a call with a bias takes the materialized implementation)");
+  if (P.D > 256 || P.Dv > 256)
+    return fail(SDPA_ERR_UNSUPPORTED, "head sizes dqk=%d dv=%d exceed the gradient kernels' limit (256)", P.D, P.Dv);
+  st = check_workspace(ws, ws_bytes, sdpa_backward_workspace_size(p));
+  if (st != SDPA_OK) return st;
+  if ((long long)P.B * P.Lq * P.H == 0 && (long long)P.B * P.Lk * P.Hkv == 0) return SDPA_OK;
+  if (!q || !k || !v || !out || !dout || !dq || !dk || !dv)
+    return fail(SDPA_ERR_INVALID_ARG, "q, k, v, out, dout, dq, dk and dv must not be NULL");
+  P.status = static_cast<int*>(ws);
+  cudaError_t e = sdpa::launch_backward(P, q, k, v, out, dout, dq, dk, dv, dscale,
+                                        static_cast<char*>(ws) + kStatusBytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gradient launch");
+  g_last_kernel = "backward_simt";
+  return SDPA_OK;
+}
+
 sdpa_status cache_update_at_index(void* k_cache, void* v_cache, const void* k_new,
                                   const void* v_new, sdpa_dtype dtype, int32_t d,
                                   int32_t nkvheads, int32_t n_new, int32_t capacity,

@@ -108,7 +108,10 @@ typedef struct sdpa_block_mask_info {
  *                   causal == SDPA_CAUSAL_TOP_LEFT.
  *  q_lengths, kv_lengths   device int32[batch] or NULL (full length). Keys j >= kv_lengths[b]
  *                   are not attended; output rows i >= q_lengths[b] are zero. Values must
- *                   lie in [0, q_len] / [0, kv_len].
+ *                   lie in [0, q_len] / [0, kv_len]. The tcgen05 kernel reads whole tiles of
+ *                   128 keys, so the rows of k and v past kv_lengths[b], up to the next
+ *                   multiple of 128 (or the array end), must hold finite values: they get a
+ *                   weight of exactly 0, and 0 times Inf or NaN is NaN.
  *  bias             NULL or a device array of bias_dtype, element (key j, query i, head h,
  *                   batch b) at bias[j*bias_stride[0] + i*bias_stride[1] + h*bias_stride[2]
  *                   + b*bias_stride[3]]; a stride of 0 broadcasts (argument `bias`: added to
@@ -152,6 +155,71 @@ SDPA_API sdpa_status sdpa_workspace_init(void* ws, size_t ws_bytes, struct CUstr
  * gives NaN (section "Fused implementation"). Returns SDPA_OK once the work is enqueued. */
 SDPA_API sdpa_status sdpa_forward(const sdpa_params* p, const void* q, const void* k, const void* v,
                          void* out, void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* Packed sequences (keywords q_segments, kv_segments and maxlen, paragraph "Packed
+ * sequences"): nseg sequences stored one after the other along the sequence axis, with no
+ * batch axis and no padding.
+ *  q_segments   device int32[nseg]: the length of each query sequence.
+ *  kv_segments  device int32[nseg]: the length of each key/value sequence, or NULL to reuse
+ *               q_segments (the keyword's default).
+ *  maxlen       at least every entry of both arrays. The host never reads the lengths: the
+ *               work is sized by nseg and maxlen. A segment longer than maxlen is an error,
+ *               found on the device. */
+typedef struct sdpa_packed_segments {
+  int32_t nseg;
+  int32_t maxlen;
+  const int32_t* q_segments;
+  const int32_t* kv_segments;
+} sdpa_packed_segments;
+
+/* Workspace bytes sdpa_forward_packed needs (256-byte aligned; 0 if the arguments are
+ * invalid). */
+SDPA_API size_t sdpa_packed_workspace_size(const sdpa_params* p, const sdpa_packed_segments* seg);
+
+/* scaled_dot_product_attention on packed sequences. The s-th query sequence attends to the
+ * s-th key/value sequence only, as batch element s of a padded batch would. is_causal applies
+ * within each sequence.
+ *  - Layout. q [total_q][nheads][dqk], k [total_kv][nkvheads][dqk], v [total_kv][nkvheads][dv],
+ *    out [total_q][nheads][dv]: the page's (head_dim, nheads, total_len). In p: batch = 1,
+ *    q_len = total_q, kv_len = total_kv.
+ *  - q_offset, q_lengths and kv_lengths, when given, are device int32[nseg], one entry per
+ *    sequence. q_lengths[s] and kv_lengths[s] lie in [0, segment length].
+ *  - bias, mask and block_info must be NULL (the page supports neither with segments):
+ *    SDPA_ERR_INVALID_ARG otherwise.
+ *  - Device-side checks. These set SDPA_ERR_DEVICE_CHECK in the status word:
+ *      - lengths that are negative;
+ *      - lengths above maxlen;
+ *      - lengths that do not add up to total_q / total_kv.
+ *    Rows are clamped to the arrays whatever the lengths. Rows of a sequence past maxlen are
+ *    not computed.
+ *  - Kernels. A one-block kernel first turns the lengths into the first row of each sequence
+ *    (in the workspace). The attention kernel then runs: tcgen05 for bf16/f16 with
+ *    dqk = dv = 64 or 128, the SIMT kernel otherwise. */
+SDPA_API sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed_segments* seg,
+                                         const void* q, const void* k, const void* v, void* out,
+                                         void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* Workspace bytes sdpa_backward needs for these params (256-byte aligned; 0 if invalid). */
+SDPA_API size_t sdpa_backward_workspace_size(const sdpa_params* p);
+
+/* The gradient of the fused implementation (paragraph "Fused implementation"), with respect
+ * to query, key, value and scale, for the loss sum(dout * out). The weights are recomputed
+ * from q and k and never materialized.
+ *  - Inputs. q, k, v and p are those of the sdpa_forward call that produced `out`. dout has
+ *    out's shape. All are device arrays of p->dtype.
+ *  - Outputs. dq, dk and dv (device, caller-owned) get the shapes and dtype of q, k and v. A
+ *    key/value head sums the contributions of the query heads that share it. dscale is a
+ *    device float or NULL.
+ *  - Rows that take no part. A query that attends to no key (NaN output) and a query past
+ *    q_lengths (zero output) get dq = 0 and add nothing to dk, dv or dscale.
+ *  - Arguments. mask, block_info, is_causal, q_offset, q_lengths and kv_lengths are as in
+ *    sdpa_forward. A bias is SDPA_ERR_INVALID_ARG: the page's automatic differentiation
+ *    takes the materialized implementation for a call with a bias. Head sizes are up to 256.
+ *  - Kernels. Three SIMT kernels run, fp32 throughout: per-row log-sum-exp and
+ *    delta = dout . out; dq, with dscale; then dk and dv. */
+SDPA_API sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, const void* v,
+                                   const void* out, const void* dout, void* dq, void* dk, void* dv,
+                                   float* dscale, void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
 /* Decoding with a KV cache (the page's example "decoding with a KV cache"; the Keras issue
  * "MultiHeadAttention is missing a position_bias call argument", cache_update_index):
@@ -227,8 +295,9 @@ SDPA_API sdpa_status sdpa_read_device_status(void* ws, struct CUstream_st* strea
 /* Message for the last non-OK status returned on this host thread. */
 SDPA_API const char* sdpa_last_error(void);
 
-/* Name of the kernel the last sdpa_forward / sdpa_decode_with_cache call on this host thread
- * launched for its attention ("generic_simt", "prefill_tcgen05", "decode_splitkv"). */
+/* Name of the kernel the last sdpa_forward / sdpa_forward_packed / sdpa_decode_with_cache /
+ * sdpa_backward call on this host thread launched for its attention ("generic_simt",
+ * "prefill_tcgen05", "decode_splitkv", "backward_simt"). */
 SDPA_API const char* sdpa_last_kernel(void);
 
 #ifdef __cplusplus

@@ -48,6 +48,9 @@ class Workload:
     p_empty: float = 0.0
     p_full: float = 0.0
     p_partial: float = 0.0
+    # packed sequences only: sequence lengths drawn uniformly from [seg_min, seg_max]
+    seg_min: int = 0
+    seg_max: int = 0
 
 
 # The five workloads of the benchmark plan, with the sizes they are quoted on.
@@ -68,7 +71,14 @@ BLOCK_SPARSE = Workload("block_sparse_mask_bf16_b1_h16_d128_l16384", batch=1, q_
                         causal=False, seed=5, block=128, p_empty=0.5, p_full=0.3,
                         p_partial=0.2)
 
-ALL = (TINY_FP32, CAUSAL_GQA_PREFILL, KV_CACHE_DECODE, ALIBI_T5_BIAS, BLOCK_SPARSE)
+# Documents of 64 to 4096 positions packed into 65536 positions (keywords q_segments /
+# kv_segments; the heads and head size of the causal GQA prefill). q_len / kv_len are the
+# packed totals; batch is unused.
+PACKED_DOCS = Workload("packed_docs_causal_gqa_bf16_h32kv8_d128_t65536", batch=1, q_len=65536,
+                       kv_len=65536, nheads=32, nkvheads=8, head_dim=128, dtype="bf16",
+                       causal=True, seed=6, seg_min=64, seg_max=4096)
+
+ALL = (TINY_FP32, CAUSAL_GQA_PREFILL, KV_CACHE_DECODE, ALIBI_T5_BIAS, BLOCK_SPARSE, PACKED_DOCS)
 
 
 def scaled(w: Workload, **changes) -> Workload:
@@ -211,3 +221,23 @@ def mask_device(w: Workload, cls: np.ndarray, device) -> torch.Tensor:
             row = torch.where(diag, torch.ones_like(row), row)
             out[h, i0:i0 + len(i)] = row
     return out
+
+
+def packed_segments(w: Workload) -> list:
+    """Sequence lengths, uniform in [seg_min, seg_max], adding up to w.q_len (the last one is
+    cut to fit)."""
+    rng = rng_for(w.seed + 1)
+    segs, total = [], 0
+    while total < w.q_len:
+        n = int(min(rng.integers(w.seg_min, w.seg_max + 1), w.q_len - total))
+        segs.append(n)
+        total += n
+    return segs
+
+
+def packed_qkv(w: Workload):
+    """q (total, nheads, head_dim), k and v (total, nkvheads, head_dim), i.i.d. N(0, 1)."""
+    rng = rng_for(w.seed)
+    return (normal(rng, (w.q_len, w.nheads, w.head_dim), w.dtype),
+            normal(rng, (w.kv_len, w.nkvheads, w.head_dim), w.dtype),
+            normal(rng, (w.kv_len, w.nkvheads, w.head_dim), w.dtype))

@@ -32,11 +32,14 @@ def test_struct_layout_matches_binding(tmp_path):
     src = tmp_path / "layout.c"
     fields = [f[0] for f in sdpa.Params._fields_]
     bfields = [f[0] for f in sdpa.BlockMaskInfoStruct._fields_]
+    sfields = [f[0] for f in sdpa.PackedSegments._fields_]
     body = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', 'int main(void){']
     body.append('printf("%zu\\n", sizeof(sdpa_params));')
     body += [f'printf("%zu\\n", offsetof(sdpa_params, {f}));' for f in fields]
     body.append('printf("%zu\\n", sizeof(sdpa_block_mask_info));')
     body += [f'printf("%zu\\n", offsetof(sdpa_block_mask_info, {f}));' for f in bfields]
+    body.append('printf("%zu\\n", sizeof(sdpa_packed_segments));')
+    body += [f'printf("%zu\\n", offsetof(sdpa_packed_segments, {f}));' for f in sfields]
     body.append('return 0;}')
     src.write_text("\n".join(body))
     exe = tmp_path / "layout"
@@ -44,6 +47,7 @@ def test_struct_layout_matches_binding(tmp_path):
     got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
     want = [ctypes.sizeof(sdpa.Params)] + [getattr(sdpa.Params, f).offset for f in fields]
     want += [ctypes.sizeof(sdpa.BlockMaskInfoStruct)] + [getattr(sdpa.BlockMaskInfoStruct, f).offset for f in bfields]
+    want += [ctypes.sizeof(sdpa.PackedSegments)] + [getattr(sdpa.PackedSegments, f).offset for f in sfields]
     assert got == want
 
 
@@ -136,3 +140,57 @@ def test_block_info_must_match_the_call():
     p = _params(block_info=ctypes.pointer(st))
     assert _forward(p) == sdpa.SDPA_ERR_INVALID_ARG
     assert "block_info" in sdpa.lib.sdpa_last_error().decode()
+
+
+def _packed_call(p, seg, ws=FAKE, ws_bytes=1 << 30):
+    return sdpa.lib.sdpa_forward_packed(ctypes.byref(p), None if seg is None else ctypes.byref(seg),
+                                        FAKE, FAKE, FAKE, FAKE, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("pkw,skw,words", [
+    (dict(batch=2), dict(), "batch must be 1"),
+    (dict(bias=FAKE, bias_dtype=sdpa.SDPA_BF16), dict(), "not supported"),
+    (dict(mask=FAKE), dict(), "not supported"),
+    (dict(), dict(nseg=-1), "negative"),
+    (dict(), dict(maxlen=-3), "negative"),
+    (dict(), dict(q_segments=None), "q_segments is NULL"),
+    (dict(), dict(nseg=0), "no segments"),
+])
+def test_packed_argument_rules(pkw, skw, words):
+    """Packed sequences: no batch axis, no bias or mask, a segment vector for any rows."""
+    p = _params(**{**dict(batch=1, q_len=300, kv_len=300), **pkw})
+    seg = sdpa.PackedSegments(3, 200, FAKE, None)
+    for k, v in skw.items():
+        setattr(seg, k, v)
+    assert _packed_call(p, seg) == sdpa.SDPA_ERR_INVALID_ARG
+    assert words in sdpa.lib.sdpa_last_error().decode()
+    assert sdpa.lib.sdpa_packed_workspace_size(ctypes.byref(p), ctypes.byref(seg)) == 0
+
+
+def test_packed_workspace_holds_the_segment_starts():
+    p = _params(batch=1, q_len=300, kv_len=300)
+    assert _packed_call(p, None) == sdpa.SDPA_ERR_INVALID_ARG
+    for nseg in (1, 63, 64, 5000):
+        seg = sdpa.PackedSegments(nseg, 300, FAKE, None)
+        need = sdpa.lib.sdpa_packed_workspace_size(ctypes.byref(p), ctypes.byref(seg))
+        assert need % 256 == 0 and need >= 256 + 2 * 4 * (nseg + 1)
+        assert _packed_call(p, seg, ws_bytes=need - 1) == sdpa.SDPA_ERR_WORKSPACE
+
+
+def test_backward_argument_rules():
+    """The fused gradient takes no bias and head sizes up to 256; its workspace holds two floats
+    per query row and head."""
+    p = _params(bias=FAKE, bias_dtype=sdpa.SDPA_BF16)
+    rc = sdpa.lib.sdpa_backward(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                1 << 30, None)
+    assert rc == sdpa.SDPA_ERR_INVALID_ARG and "bias" in sdpa.lib.sdpa_last_error().decode()
+    p = _params(dqk=320, dv=64)
+    rc = sdpa.lib.sdpa_backward(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                1 << 30, None)
+    assert rc == sdpa.SDPA_ERR_UNSUPPORTED
+    p = _params(batch=4, q_len=2048, nheads=32, nkvheads=8)
+    need = sdpa.lib.sdpa_backward_workspace_size(ctypes.byref(p))
+    assert need % 256 == 0 and need >= 256 + 4 * 2048 * 32 * 8
+    rc = sdpa.lib.sdpa_backward(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                need - 1, None)
+    assert rc == sdpa.SDPA_ERR_WORKSPACE
