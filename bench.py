@@ -401,7 +401,9 @@ def packed_workload(args, dev, world, ws, peaks):
 
 def backward_workload(args, dev, world, ws, peaks):
     """The fused gradient (dq, dk, dv, dscale) of the causal GQA prefill workload: 10*head_dim
-    flops per attended pair (the logits recomputed, dout.v, and the dv, dq and dk products)."""
+    flops per attended pair (the logits recomputed, dout.v, and the dv, dq and dk products;
+    the tiled kernels also recompute the logits once more for the row log-sum-exp, which is
+    not counted)."""
     import head_scaled_dot_sdpa_b200 as sdpa
 
     w = si.CAUSAL_GQA_PREFILL
@@ -417,7 +419,7 @@ def backward_workload(args, dev, world, ws, peaks):
             "ms_per_step": round(ms, 3), "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
                          "frac": round(tf / peaks["bf16"], 5)},
-            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 3}
+            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 2 if sdpa.last_kernel() == "backward_mma" else 3}
 
 
 # ---- CPU oracle ---------------------------------------------------------------------------------

@@ -273,7 +273,8 @@ def sdpa_forward(q, k, v, bias=None, *, mask=None, scale=None, is_causal=False, 
 
 
 def sdpa_backward(q, k, v, out, dout, *, mask=None, scale=None, is_causal=False, q_offset=0,
-                  q_lengths=None, kv_lengths=None, block_info=None, workspace=None, stream=None):
+                  q_lengths=None, kv_lengths=None, block_info=None, workspace=None, generic=False,
+                  stream=None):
     """The gradient of the fused implementation for the loss sum(dout * out), where `out` is
     sdpa_forward(q, k, v; ...) with the same arguments: returns (dq, dk, dv, dscale), dscale a
     0-d float32 device tensor. Rows with no attended key and rows past q_lengths take no part.
@@ -284,7 +285,8 @@ def sdpa_backward(q, k, v, out, dout, *, mask=None, scale=None, is_causal=False,
             raise ValueError(f"{n} must be a contiguous CUDA tensor of the output's shape and dtype")
     keep = []
     p = _params(q, k, v, bias=None, mask=mask, scale=scale, is_causal=is_causal, q_offset=q_offset,
-                q_lengths=q_lengths, kv_lengths=kv_lengths, block_info=block_info, flags=0, keep=keep)
+                q_lengths=q_lengths, kv_lengths=kv_lengths, block_info=block_info,
+                flags=SDPA_FLAG_GENERIC_KERNEL if generic else 0, keep=keep)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dscale = torch.zeros((), dtype=torch.float32, device=q.device)
     need = _lib.sdpa_backward_workspace_size(ctypes.byref(p))

@@ -88,6 +88,12 @@ size_t backward_workspace_bytes(const Problem& P);
 cudaError_t launch_backward(const Problem& P, const void* q, const void* k, const void* v, const void* out,
                             const void* dout, void* dq, void* dk, void* dv, float* dscale, void* ws,
                             cudaStream_t stream);
+// The same on mma.sync tiles (bf16 / fp16, head_dim = v_head_dim = 64 or 128); same workspace.
+bool backward_mma_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out,
+                            const void* dout);
+cudaError_t launch_backward_mma(const Problem& P, const void* q, const void* k, const void* v, const void* out,
+                                const void* dout, void* dq, void* dk, void* dv, float* dscale, void* ws,
+                                cudaStream_t stream);
 bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v,
                        const void* out);
 size_t prefill_workspace_bytes(const Problem& P);

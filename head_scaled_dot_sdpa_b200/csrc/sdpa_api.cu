@@ -286,8 +286,14 @@ sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, co
   if (!q || !k || !v || !out || !dout || !dq || !dk || !dv)
     return fail(SDPA_ERR_INVALID_ARG, "q, k, v, out, dout, dq, dk and dv must not be NULL");
   P.status = static_cast<int*>(ws);
-  cudaError_t e = sdpa::launch_backward(P, q, k, v, out, dout, dq, dk, dv, dscale,
-                                        static_cast<char*>(ws) + kStatusBytes, (cudaStream_t)stream);
+  void* scratch = static_cast<char*>(ws) + kStatusBytes;
+  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && sdpa::backward_mma_supported(P, q, k, v, out, dout)) {
+    cudaError_t e = sdpa::launch_backward_mma(P, q, k, v, out, dout, dq, dk, dv, dscale, scratch, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gradient launch");
+    g_last_kernel = "backward_mma";
+    return SDPA_OK;
+  }
+  cudaError_t e = sdpa::launch_backward(P, q, k, v, out, dout, dq, dk, dv, dscale, scratch, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "gradient launch");
   g_last_kernel = "backward_simt";
   return SDPA_OK;

@@ -215,8 +215,10 @@ SDPA_API size_t sdpa_backward_workspace_size(const sdpa_params* p);
  *  - Arguments. mask, block_info, is_causal, q_offset, q_lengths and kv_lengths are as in
  *    sdpa_forward. A bias is SDPA_ERR_INVALID_ARG: the page's automatic differentiation
  *    takes the materialized implementation for a call with a bias. Head sizes are up to 256.
- *  - Kernels. Three SIMT kernels run, fp32 throughout: per-row log-sum-exp and
- *    delta = dout . out; dq, with dscale; then dk and dv. */
+ *  - Kernels. bf16/fp16 with dqk = dv = 64 or 128 run two mma.sync tile kernels: dq (with the
+ *    row log-sum-exp, delta = dout . out and dscale), then dk and dv per key tile. dscale is
+ *    zeroed first with cudaMemsetAsync. Other types and sizes, or SDPA_FLAG_GENERIC_KERNEL,
+ *    take three SIMT kernels, fp32 throughout. */
 SDPA_API sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, const void* v,
                                    const void* out, const void* dout, void* dq, void* dk, void* dv,
                                    float* dscale, void* ws, size_t ws_bytes, struct CUstream_st* stream);

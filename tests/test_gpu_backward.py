@@ -41,13 +41,19 @@ def _inputs(seed, B, Lq, Lk, H, Hkv, D, Dv, dtype):
             si.normal(rng, (B, Lk, Hkv, Dv), n), si.normal(rng, (B, Lq, H, Dv), n))
 
 
-def check(q, k, v, dout, what, **kw):
+def expected_kernel(q, v, generic=False):
+    """mma.sync tiles for 16-bit types with head_dim = v_head_dim = 64 or 128, SIMT otherwise."""
+    tiles = q.dtype in (torch.bfloat16, torch.float16) and q.shape[-1] == v.shape[-1] in (64, 128)
+    return "backward_mma" if tiles and not generic else "backward_simt"
+
+
+def check(q, k, v, dout, what, generic=False, **kw):
     """Forward on the GPU, then the gradient on the GPU, against the oracle's gradient."""
     dt = q.dtype
     qd, kd, vd, dd = (t.to(DEV) for t in (q, k, v, dout))
     out = sdpa.sdpa_forward(qd, kd, vd, **kw)
-    dq, dk, dv, ds = sdpa.sdpa_backward(qd, kd, vd, out, dd, **kw)
-    assert sdpa.last_kernel() == "backward_simt"
+    dq, dk, dv, ds = sdpa.sdpa_backward(qd, kd, vd, out, dd, generic=generic, **kw)
+    assert sdpa.last_kernel() == expected_kernel(q, v, generic)
     assert sdpa.read_device_status() == sdpa.SDPA_OK
     okw = {a: b for a, b in kw.items() if a != "block_info"}
     if "mask" in okw:
@@ -65,10 +71,13 @@ def check(q, k, v, dout, what, **kw):
 
 
 SHAPES = [
-    # B, Lq, Lk, H, Hkv, D, Dv
+    # B, Lq, Lk, H, Hkv, D, Dv: ragged tails of the 64-query, 64-key and 32-query tiles,
+    # several tiles, GQA groups of 1 to 4
     (2, 37, 45, 4, 2, 64, 64),
     (1, 130, 200, 2, 1, 128, 128),
     (2, 64, 33, 3, 3, 40, 24),
+    (1, 200, 131, 8, 2, 128, 128),
+    (2, 97, 97, 3, 1, 64, 64),
 ]
 
 
@@ -81,7 +90,14 @@ def test_backward_shapes(dtype, shape, causal):
     check(q, k, v, dout, f"{shape} causal={causal}", is_causal=causal)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_simt_forced(causal):
+    """The SIMT kernels on a shape the tiles also take, so both paths stay covered."""
+    q, k, v, dout = _inputs(8, 1, 100, 90, 4, 2, 128, 128, torch.bfloat16)
+    check(q, k, v, dout, f"forced SIMT causal={causal}", generic=True, is_causal=causal)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 def test_backward_lengths_offsets_and_empty_rows(dtype):
     """Per-batch q_offset, q_lengths and kv_lengths, with a sequence of no keys (NaN rows, no
     part in the gradient) and padding rows."""
