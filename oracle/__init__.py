@@ -66,6 +66,9 @@ def load(path: str | None = None):
         lib = ctypes.CDLL(lib_path)
         lib.oracle_sdpa_forward.argtypes = [ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p]
         lib.oracle_sdpa_forward.restype = ctypes.c_int
+        lib.oracle_sdpa_forward_with_weights.argtypes = [
+            ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_uint64, _f64p, _f64p]
+        lib.oracle_sdpa_forward_with_weights.restype = ctypes.c_int
         lib.oracle_sdpa_backward.argtypes = [
             ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p]
         lib.oracle_sdpa_backward.restype = ctypes.c_int
@@ -183,6 +186,57 @@ def sdpa_forward(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_o
     if rc != 0:
         raise OracleError(f"oracle_sdpa_forward failed with code {rc}")
     return out
+
+
+def sdpa_forward_with_weights(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_offset=0,
+                              q_lengths=None, kv_lengths=None, drop_p=0.0, seed=0, lib=None):
+    """scaled_dot_product_attention_with_weights(query, key, value, [bias]; fdrop, mask, scale,
+    is_causal, q_offset, q_lengths, kv_lengths) in float64, with fdrop = dropout of probability
+    drop_p drawn by the counter-based generator of the C source (seeded by `seed`). Returns
+    (out (B, Lq, H, dv), weights (B, H, Lq, Lk)): the weights after the dropout, the page's
+    (kv_len, q_len, nheads, batch) order."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Lq, H, D = q.shape
+    Bk, Lk, Hkv, Dk = k.shape
+    Dv = v.shape[3]
+    if Bk != B or v.shape[:3] != (B, Lk, Hkv) or Dk != D:
+        raise ValueError("inconsistent q/k/v shapes")
+    p = _Problem()
+    p.batch, p.q_len, p.kv_len, p.nheads, p.nkvheads, p.dqk, p.dv = B, Lq, Lk, H, Hkv, D, Dv
+    p.scale = float("nan") if scale is None else float(scale)
+    p.causal = {False: 0, True: 1, "bottom_right": 2}[is_causal]
+    keep = []
+    qo = np.asarray(q_offset, dtype=np.int64)
+    if qo.ndim == 0:
+        p.q_offset_scalar = int(qo)
+    else:
+        qo = _per_batch(qo, B)
+        keep.append(qo)
+        p.q_offset = _ptr(qo, _i64p)
+    for name, val in (("q_lengths", q_lengths), ("kv_lengths", kv_lengths)):
+        arr = _per_batch(val, B)
+        if arr is not None:
+            keep.append(arr)
+            setattr(p, name, _ptr(arr, _i64p))
+    if bias is not None:
+        base, st = _broadcast4(bias, np.float64, B, H, Lq, Lk)
+        keep.append(base)
+        p.bias = _ptr(base, _f64p)
+        p.bias_stride = (ctypes.c_int64 * 4)(*st)
+    if mask is not None:
+        base, st = _broadcast4(np.asarray(mask).astype(np.uint8), np.uint8, B, H, Lq, Lk)
+        keep.append(base)
+        p.mask = _ptr(base, _u8p)
+        p.mask_stride = (ctypes.c_int64 * 4)(*st)
+    out = np.empty((B, Lq, H, Dv), dtype=np.float64)
+    weights = np.empty((B, H, Lq, Lk), dtype=np.float64)
+    rc = lib.oracle_sdpa_forward_with_weights(ctypes.byref(p), _ptr(q, _f64p), _ptr(k, _f64p),
+                                              _ptr(v, _f64p), float(drop_p), int(seed) & (2**64 - 1),
+                                              _ptr(out, _f64p), _ptr(weights, _f64p))
+    if rc != 0:
+        raise OracleError(f"oracle_sdpa_forward_with_weights failed with code {rc}")
+    return out, weights
 
 
 def sdpa_backward(q, k, v, dout, mask=None, scale=None, is_causal=False, q_offset=0,

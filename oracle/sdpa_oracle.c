@@ -185,6 +185,103 @@ int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const dou
   return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
+/* Counter-based uniform draw for dropout: the 64-bit finalizer of Austin Appleby's MurmurHash3
+ * ("fmix64"), applied twice, to the element's linear index (b, h, i, j) and then to that plus
+ * the seed. The top 53 bits give u in [0, 1). */
+static uint64_t fmix64(uint64_t k) {
+  k ^= k >> 33;
+  k *= 0xff51afd7ed558ccdULL;
+  k ^= k >> 33;
+  k *= 0xc4ceb9fe1a85ec53ULL;
+  k ^= k >> 33;
+  return k;
+}
+static double dropout_uniform(uint64_t seed, uint64_t index) {
+  return (double)(fmix64(seed + fmix64(index)) >> 11) * (1.0 / 9007199254740992.0);
+}
+
+/* scaled_dot_product_attention_with_weights (the entry's "See also": the attention weights too)
+ * with an fdrop that is dropout of probability drop_p (argument fdrop: applied to the weights
+ * right after the softmax). The weights are materialized (paragraph "Fused implementation":
+ * any call with an fdrop takes the materialized implementation):
+ *   w_ij = softmax_j(scale q_i.k_j + bias_ij, masked)
+ *   w'_ij = w_ij / (1 - drop_p) where u(seed, b, h, i, j) >= drop_p, else 0
+ *   out_i = sum_j w'_ij v_j
+ * and `weights` receives w' in the page's (kv_len, q_len, nheads, batch) order, which is
+ * row-major [batch][nheads][q_len][kv_len]. A row with no attended key has NaN weights and a
+ * NaN output; a row past q_lengths has zero weights and a zero output. drop_p must be in
+ * [0, 1). */
+int oracle_sdpa_forward_with_weights(const oracle_sdpa_problem* p, const double* q, const double* k,
+                                     const double* v, double drop_p, uint64_t seed, double* out,
+                                     double* weights) {
+  int rc = check_problem(p);
+  if (rc) return rc;
+  if (!(drop_p >= 0.0 && drop_p < 1.0)) return ORACLE_ERR_ARG;
+  const int64_t B = p->batch, Lq = p->q_len, Lk = p->kv_len, H = p->nheads, Hkv = p->nkvheads;
+  const int64_t D = p->dqk, Dv = p->dv, group = H / Hkv;
+  const double scale = isnan(p->scale) ? 1.0 / sqrt((double)D) : p->scale;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t r = 0; r < B * H * Lq; ++r) {
+    const int64_t b = r / (H * Lq), h = (r / Lq) % H, i = r % Lq;
+    double* wrow = weights + ((b * H + h) * Lq + i) * Lk;
+    double* o = out + ((b * Lq + i) * H + h) * Dv;
+    const int64_t qlen_b = p->q_lengths ? p->q_lengths[b] : Lq;
+    const int64_t kvlen_b = p->kv_lengths ? p->kv_lengths[b] : Lk;
+    for (int64_t j = 0; j < Lk; ++j) wrow[j] = 0.0;
+    for (int64_t e = 0; e < Dv; ++e) o[e] = 0.0;
+    if (i >= qlen_b) continue;
+    int64_t off = 0;
+    if (p->causal == 1) off = p->q_offset ? p->q_offset[b] : p->q_offset_scalar;
+    if (p->causal == 2) off = kvlen_b - qlen_b;
+    const int64_t g = h / group;
+    const double* qi = q + ((b * Lq + i) * H + h) * D;
+    double m = -INFINITY;
+    int64_t n = 0;
+    for (int64_t j = 0; j < Lk; ++j) {
+      int a = (j < kvlen_b);
+      if (p->causal != 0 && !(j <= off + i)) a = 0;
+      if (p->mask && !p->mask[j * p->mask_stride[0] + i * p->mask_stride[1] + h * p->mask_stride[2] +
+                              b * p->mask_stride[3]])
+        a = 0;
+      if (!a) {
+        wrow[j] = -INFINITY;
+        continue;
+      }
+      const double* kj = k + ((b * Lk + j) * Hkv + g) * D;
+      double dot = 0.0;
+      for (int64_t c = 0; c < D; ++c) dot += qi[c] * kj[c];
+      double x = scale * dot;
+      if (p->bias)
+        x += p->bias[j * p->bias_stride[0] + i * p->bias_stride[1] + h * p->bias_stride[2] +
+                     b * p->bias_stride[3]];
+      wrow[j] = x;
+      if (x > m) m = x;
+      ++n;
+    }
+    if (n == 0) {
+      for (int64_t j = 0; j < Lk; ++j) wrow[j] = NAN;
+      for (int64_t e = 0; e < Dv; ++e) o[e] = NAN;
+      continue;
+    }
+    double z = 0.0;
+    for (int64_t j = 0; j < Lk; ++j) {
+      wrow[j] = (wrow[j] == -INFINITY) ? 0.0 : exp(wrow[j] - m);
+      z += wrow[j];
+    }
+    const uint64_t base = (uint64_t)(((b * H + h) * Lq + i) * Lk);
+    for (int64_t j = 0; j < Lk; ++j) {
+      double w = wrow[j] / z;
+      if (drop_p > 0.0)
+        w = (dropout_uniform(seed, base + (uint64_t)j) >= drop_p) ? w / (1.0 - drop_p) : 0.0;
+      wrow[j] = w;
+      if (w == 0.0) continue;
+      const double* vj = v + ((b * Lk + j) * Hkv + g) * Dv;
+      for (int64_t e = 0; e < Dv; ++e) o[e] += w * vj[e];
+    }
+  }
+  return ORACLE_OK;
+}
+
 /* The gradient of the fused implementation (paragraph "Fused implementation": the fused
  * implementation has a gradient with respect to query, key, value and scale, and a query that
  * attends to no key, whose output is NaN, takes no part in it). For the loss

@@ -382,6 +382,80 @@ def printed_example_shapes(lib):
         assert np.isfinite(out).all()
 
 
+# ---- with weights and fdrop (the entry's "See also"; argument fdrop) -------------------------
+
+@pin
+def with_weights_equals_torch_softmax(lib):
+    """The materialized weights are PyTorch's float64 softmax of scale*q.k + bias over the
+    attended keys (masked logits at -inf; GQA by repeated heads), in the page's (kv_len,
+    q_len, nheads, batch) order, and the output is those weights times V."""
+    rng = _rng(81)
+    q, k, v = _qkv(rng, 2, 5, 7, 4, 2, 6, 3)
+    bias = rng.standard_normal((4, 5, 7))
+    mask = rng.random((2, 4, 5, 7)) < 0.7
+    mask[..., 0] = True
+    out, w = oracle.sdpa_forward_with_weights(q, k, v, bias=bias, mask=mask, scale=0.6, lib=lib)
+    kk = np.repeat(k, 2, axis=2)
+    logits = 0.6 * np.einsum("bihc,bjhc->bhij", q, kk) + bias[None]
+    logits = torch.from_numpy(np.where(mask, logits, -np.inf))
+    want = torch.softmax(logits, dim=-1).numpy()
+    _close(w, want)
+    _close(out, np.einsum("bhij,bjhe->bihe", w, np.repeat(v, 2, axis=2)))
+
+
+@pin
+def with_weights_empty_and_padding_rows(lib):
+    """A row with no attended key has NaN weights and output; a row past q_lengths has zero
+    weights and output; causal rows put no weight past q_offset + i."""
+    rng = _rng(82)
+    q, k, v = _qkv(rng, 2, 4, 6, 2, 2, 4)
+    out, w = oracle.sdpa_forward_with_weights(q, k, v, is_causal=True, q_offset=[1, -2],
+                                              q_lengths=[3, 4], lib=lib)
+    assert np.isnan(w[1, :, :2]).all() and np.isnan(out[1, :2]).all()
+    assert (w[0, :, 3] == 0).all() and (out[0, 3] == 0).all()
+    i = np.arange(4)[:, None]
+    j = np.arange(6)[None, :]
+    # softmax weights are positive exactly on the attended keys j <= q_offset + i
+    assert ((w[0, :, :3] > 0) == (j <= 1 + i)[None, :3]).all()
+    assert ((w[1, :, 2:] > 0) == (j <= -2 + i)[None, 2:]).all()
+    _close(np.nansum(w[0, :, :3], axis=-1), np.ones((2, 3)))
+
+
+@pin
+def dropout_keeps_one_minus_p_unbiased(lib):
+    """fdrop as dropout: each weight is kept with probability 1 - p and then divided by 1 - p,
+    so the kept fraction is 1 - p (checked within 5 standard deviations on 40,000 weights) and
+    the average over seeds is the undropped weight. The output is the dropped weights times
+    V. p = 0 changes nothing; another seed gives another pattern."""
+    rng = _rng(83)
+    q, k, v = _qkv(rng, 2, 40, 50, 10, 5, 8)
+    o0, w0 = oracle.sdpa_forward_with_weights(q, k, v, lib=lib)
+    o1, w1 = oracle.sdpa_forward_with_weights(q, k, v, drop_p=0.0, seed=99, lib=lib)
+    _close(w0, w1, 0.0)
+    _close(o0, o1, 0.0)
+    p = 0.3
+    out, w = oracle.sdpa_forward_with_weights(q, k, v, drop_p=p, seed=7, lib=lib)
+    kept = w != 0
+    n = kept.size
+    assert abs(kept.mean() - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
+    _close(w[kept], w0[kept] / (1 - p), 1e-15)
+    _close(out, np.einsum("bhij,bjhe->bihe", w, np.repeat(v, 2, axis=2)))
+    _, w2 = oracle.sdpa_forward_with_weights(q, k, v, drop_p=p, seed=8, lib=lib)
+    assert ((w2 != 0) != kept).mean() > 0.3
+    acc = np.zeros((1, 10, 4, 50))
+    for s in range(300):
+        acc += oracle.sdpa_forward_with_weights(q[:1, :4], k[:1], v[:1], drop_p=p, seed=1000 + s, lib=lib)[1]
+    ref = w0[:1, :, :4]
+    sd = np.sqrt(ref ** 2 * p / (1 - p) / 300)
+    assert (np.abs(acc / 300 - ref) <= 5 * sd + 1e-12).all()
+    try:
+        oracle.sdpa_forward_with_weights(q, k, v, drop_p=1.0, lib=lib)
+    except oracle.OracleError:
+        pass
+    else:
+        raise AssertionError("drop probability 1 accepted")
+
+
 # ---- the fused gradient (paragraph "Fused implementation") -----------------------------------
 
 def _loss(q, k, v, dout, lib, **kw):

@@ -34,11 +34,18 @@ MUTANTS = {
     "block_class_swapped": ("(set == cells ? 2 : 1)", "(set == cells ? 1 : 2)"),
     "block_bits_reversed": ("word |= (1u << c);", "word |= (1u << (31 - c));"),
     "block_full_at_edge": ("(set == cells ? 2 : 1)", "(set == bq * bk ? 2 : 1)"),
+    "weights_dropout_unscaled": ("? w / (1.0 - drop_p) : 0.0", "? w : 0.0"),
+    "weights_dropout_inverted": ("base + (uint64_t)j) >= drop_p)", "base + (uint64_t)j) < drop_p)"),
+    "weights_head_batch_swapped": ("double* wrow = weights + ((b * H + h) * Lq + i) * Lk;",
+                                   "double* wrow = weights + ((h * B + b) * Lq + i) * Lk;"),
     "backward_delta_sign": ("x[j] * (dw[j] - wdw)", "x[j] * (dw[j] + wdw)"),
     "backward_dk_unscaled": ("dkj[c] += scale * dx * qi[c];", "dkj[c] += dx * qi[c];"),
     "backward_dv_from_dx": ("dvj[e] += x[j] * doi[e];", "dvj[e] += dx * doi[e];"),
     "backward_dscale_scaled": ("total += dx * dot;", "total += dx * dot * scale;"),
-    "backward_causal_off_by_one": ("!(j <= off + i)) a = 0;", "!(j < off + i)) a = 0;"),
+    "backward_causal_off_by_one": ("          if (p->causal != 0 && !(j <= off + i)) a = 0;",
+                                   "          if (p->causal != 0 && !(j < off + i)) a = 0;"),
+    "weights_causal_off_by_one": ("      if (p->causal != 0 && !(j <= off + i)) a = 0;",
+                                  "      if (p->causal != 0 && !(j < off + i)) a = 0;"),
     # packed mutants move starts only toward lower addresses, so every access stays in bounds
     "packed_kv_segments_ignored": ("kv_segments ? kv_segments : q_segments;", "q_segments;"),
     "packed_query_start": ("q + q0 * H * p->dqk", "q + q0 * Hkv * p->dqk"),
