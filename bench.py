@@ -286,19 +286,22 @@ def run_ours(args, rank, world, local):
 
 
 def other_workloads(args, dev, world, ws, peaks):
-    import head_scaled_dot_sdpa_b200 as sdpa
-
+    """The other rows of the hot path, each timed like the headline. A workload that raises is
+    reported as {"error": ...} so that the line with the headline is still printed."""
+    runs = (("decode", "kv_cache_decode", lambda: decode_workload(args, dev, world, ws, peaks)),
+            ("bias", "alibi_t5_bias", lambda: bias_workload(args, dev, world, ws)),
+            ("block_sparse", "block_sparse_mask", lambda: block_sparse_workload(args, dev, world, ws, peaks)),
+            ("packed", "packed_docs", lambda: packed_workload(args, dev, world, ws, peaks)),
+            ("backward", "fused_gradient", lambda: backward_workload(args, dev, world, ws, peaks)),
+            ("weights", "with_weights", lambda: weights_workload(args, dev, world, ws, peaks)))
     res = {}
-    if "decode" in args.workloads:
-        res["kv_cache_decode"] = decode_workload(args, dev, world, ws, peaks)
-    if "bias" in args.workloads:
-        res["alibi_t5_bias"] = bias_workload(args, dev, world, ws)
-    if "block_sparse" in args.workloads:
-        res["block_sparse_mask"] = block_sparse_workload(args, dev, world, ws, peaks)
-    if "packed" in args.workloads:
-        res["packed_docs"] = packed_workload(args, dev, world, ws, peaks)
-    if "backward" in args.workloads:
-        res["fused_gradient"] = backward_workload(args, dev, world, ws, peaks)
+    for key, name, run in runs:
+        if key not in args.workloads:
+            continue
+        try:
+            res[name] = run()
+        except Exception as e:  # noqa: BLE001 - reported in the JSON line
+            res[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
     return res
 
 
@@ -422,6 +425,29 @@ def backward_workload(args, dev, world, ws, peaks):
             "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 2 if sdpa.last_kernel() == "backward_mma" else 3}
 
 
+def weights_workload(args, dev, world, ws, peaks):
+    """scaled_dot_product_attention_with_weights with dropout (p = 0.1) on the causal GQA
+    workload: the whole (batch, nheads, q_len, kv_len) weight array is written, so the step is
+    bound by that write (plus reading Q, K, V and writing out)."""
+    import head_scaled_dot_sdpa_b200 as sdpa
+
+    w = si.CAUSAL_GQA_PREFILL
+    q, k, v = [t.to(dev) for t in si.qkv(w)]
+    out = torch.empty_like(q)
+    weights = torch.empty((w.batch, w.nheads, w.q_len, w.kv_len), dtype=q.dtype, device=dev)
+    byts = weights.numel() * 2 + 2 * q.numel() * 2 + 2 * k.numel() * 2
+    step = lambda: sdpa.sdpa_forward_with_weights(q, k, v, is_causal=True, drop_p=0.1, seed=1, out=out,
+                                                  weights=weights, workspace=ws)
+    per = time_steps(step, max(3, args.steps // 4), args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"workload": w.name + "_with_weights_p0.1", "metric": "HBM GB/s", "value": round(gbs * world, 1),
+            "unit": "GB/s", "ms_per_step": round(ms, 3), "bytes_per_step": byts,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm"], 4)},
+            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 1}
+
+
 # ---- CPU oracle ---------------------------------------------------------------------------------
 
 def _oracle_heads(q, k, v, heads, group):
@@ -502,7 +528,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--reference-heads", type=int, default=16)
-    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse,packed,backward",
+    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse,packed,backward,weights",
                     help="comma list; without 'prefill' only the other workloads run (a profiling aid)")
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide the decode batch and the block-sparse length by this (small ncu cases)")

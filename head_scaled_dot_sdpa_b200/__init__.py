@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "libsdpa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing; build it with `python -m head_scaled_dot_sdpa_b200.build`")
+        f"{LIB_PATH} is missing; build it with `python head_scaled_dot_sdpa_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 # ---- ABI mirror -------------------------------------------------------------------------------
@@ -78,6 +78,8 @@ _lib.sdpa_forward.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sdpa_packed_workspace_size.argtypes = [_PP, ctypes.POINTER(PackedSegments)]
 _lib.sdpa_packed_workspace_size.restype = _sz
 _lib.sdpa_forward_packed.argtypes = [_PP, ctypes.POINTER(PackedSegments), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sdpa_forward_with_weights.argtypes = [_PP, ctypes.c_double, ctypes.c_uint64, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                           _vp]
 _lib.sdpa_backward_workspace_size.argtypes = [_PP]
 _lib.sdpa_backward_workspace_size.restype = _sz
 _lib.sdpa_backward.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -91,7 +93,8 @@ _lib.build_block_mask_info.argtypes = [_vp, ctypes.POINTER(ctypes.c_int64), _i32
 _lib.sdpa_read_device_status.argtypes = [_vp, _vp]
 _lib.sdpa_last_error.restype = ctypes.c_char_p
 _lib.sdpa_last_kernel.restype = ctypes.c_char_p
-for _f in ("sdpa_workspace_init", "sdpa_forward", "sdpa_forward_packed", "sdpa_backward", "sdpa_decode_with_cache",
+for _f in ("sdpa_workspace_init", "sdpa_forward", "sdpa_forward_packed", "sdpa_forward_with_weights",
+           "sdpa_backward", "sdpa_decode_with_cache",
            "cache_update_at_index",
            "build_block_mask_info", "sdpa_read_device_status"):
     getattr(_lib, _f).restype = ctypes.c_int
@@ -270,6 +273,30 @@ def sdpa_forward(q, k, v, bias=None, *, mask=None, scale=None, is_causal=False, 
     _check(_lib.sdpa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), ws.ptr,
                              ws.nbytes, _stream(stream)))
     return out
+
+
+def sdpa_forward_with_weights(q, k, v, bias=None, *, mask=None, scale=None, is_causal=False, q_offset=0,
+                              q_lengths=None, kv_lengths=None, block_info=None, drop_p=0.0, seed=0, out=None,
+                              weights=None, workspace=None, generic=False, stream=None):
+    """scaled_dot_product_attention_with_weights(q, k, v, [bias]; fdrop, mask, scale, is_causal,
+    q_offset, q_lengths, kv_lengths), fdrop being dropout of probability drop_p with the
+    library's counter-based generator (seed). Returns (out (B, Lq, H, dv), weights (B, H, Lq,
+    Lk)), the weights after the dropout, in the page's (kv_len, q_len, nheads, batch) order."""
+    _check_qkv(q, k, v)
+    keep = []
+    p = _params(q, k, v, bias=bias, mask=mask, scale=scale, is_causal=is_causal, q_offset=q_offset,
+                q_lengths=q_lengths, kv_lengths=kv_lengths, block_info=block_info,
+                flags=SDPA_FLAG_GENERIC_KERNEL if generic else 0, keep=keep)
+    B, Lq, H, _ = q.shape
+    if out is None:
+        out = torch.empty(q.shape[:3] + (v.shape[3],), dtype=q.dtype, device=q.device)
+    if weights is None:
+        weights = torch.empty((B, H, Lq, k.shape[1]), dtype=q.dtype, device=q.device)
+    ws = _workspace(q.device, 256, workspace)
+    _check(_lib.sdpa_forward_with_weights(ctypes.byref(p), float(drop_p), int(seed) & (2**64 - 1), _ptr(q),
+                                          _ptr(k), _ptr(v), _ptr(out), _ptr(weights), ws.ptr, ws.nbytes,
+                                          _stream(stream)))
+    return out, weights
 
 
 def sdpa_backward(q, k, v, out, dout, *, mask=None, scale=None, is_causal=False, q_offset=0,
@@ -452,6 +479,6 @@ def build_block_mask_info(mask, bq: int = 128, bk: int = 128, *, stream=None) ->
     return info
 
 
-__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
+__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_forward_with_weights", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
            "build_block_mask_info", "BlockMaskInfo", "Workspace", "read_device_status",
            "last_kernel", "SdpaError", "lib"]

@@ -1,6 +1,8 @@
 """Builds libsdpa.so in-tree: every .cu under csrc/ compiled by nvcc for sm_100a only.
 
-    python -m head_scaled_dot_sdpa_b200.build [--force]
+    python head_scaled_dot_sdpa_b200/build.py [--force]
+
+(run as a file, so that the package, which loads the library, is not imported first)
 
 The CUDA runtime is linked statically and the driver API (used for TMA descriptors) is
 looked up at run time, so the library loads on a machine without a GPU driver.

@@ -94,6 +94,11 @@ bool backward_mma_supported(const Problem& P, const void* q, const void* k, cons
 cudaError_t launch_backward_mma(const Problem& P, const void* q, const void* k, const void* v, const void* out,
                                 const void* dout, void* dq, void* dk, void* dv, float* dscale, void* ws,
                                 cudaStream_t stream);
+// scaled_dot_product_attention_with_weights with dropout: mma.sync tiles (bf16 / fp16,
+// head_dim = v_head_dim = 64 or 128) or SIMT. Needs no workspace.
+bool weights_mma_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out);
+cudaError_t launch_weights(const Problem& P, bool tiles, const void* q, const void* k, const void* v, void* out,
+                           void* weights, double drop_p, unsigned long long seed, cudaStream_t stream);
 bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v,
                        const void* out);
 size_t prefill_workspace_bytes(const Problem& P);

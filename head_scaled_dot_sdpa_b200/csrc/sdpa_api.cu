@@ -263,6 +263,29 @@ sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed_segments
   return SDPA_OK;
 }
 
+sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop_p, uint64_t seed, const void* q,
+                                      const void* k, const void* v, void* out, void* weights, void* ws,
+                                      size_t ws_bytes, struct CUstream_st* stream) {
+  sdpa::Problem P;
+  sdpa_status st = resolve(p, &P);
+  if (st != SDPA_OK) return st;
+  if (!(drop_p >= 0.0 && drop_p < 1.0)) return fail(SDPA_ERR_INVALID_ARG, "drop probability %g is not in [0, 1)", drop_p);
+  if (P.Dv > 256) return fail(SDPA_ERR_UNSUPPORTED, "v_head_dim %d exceeds the weights kernels' limit (256)", P.Dv);
+  if (P.D > 1024) return fail(SDPA_ERR_UNSUPPORTED, "head_dim %d exceeds the weights kernels' limit (1024)", P.D);
+  st = check_workspace(ws, ws_bytes, kStatusBytes);
+  if (st != SDPA_OK) return st;
+  if ((long long)P.B * P.Lq * P.H == 0) return SDPA_OK;
+  if (!q || !out || !weights || (P.Lk > 0 && (!k || !v)))
+    return fail(SDPA_ERR_INVALID_ARG, "q, k, v, out and weights must not be NULL");
+  P.status = static_cast<int*>(ws);
+  const bool tiles = !(p->flags & SDPA_FLAG_GENERIC_KERNEL) && P.Lk > 0 && sdpa::weights_mma_supported(P, q, k, v, out);
+  cudaError_t e = sdpa::launch_weights(P, tiles, q, k, v, out, weights, drop_p, (unsigned long long)seed,
+                                       (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "weights launch");
+  g_last_kernel = tiles ? "weights_mma" : "weights_simt";
+  return SDPA_OK;
+}
+
 size_t sdpa_backward_workspace_size(const sdpa_params* p) {
   sdpa::Problem P;
   if (resolve(p, &P) != SDPA_OK) return 0;

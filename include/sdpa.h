@@ -199,6 +199,26 @@ SDPA_API sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed
                                          const void* q, const void* k, const void* v, void* out,
                                          void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* scaled_dot_product_attention_with_weights (the entry's "See also": the attention weights
+ * too) with fdrop as dropout of probability drop_p (argument fdrop: applied to the weights right
+ * after the softmax). The weights are materialized, as the page's materialized implementation
+ * does for such calls.
+ *  - Arguments are those of sdpa_forward, all supported, bias and mask included.
+ *  - weights (device, caller-owned, p->dtype) gets the page's (kv_len, q_len, nheads, batch)
+ *    order, row-major [batch][nheads][q_len][kv_len], after the dropout. A row with no attended
+ *    key has NaN weights and output. A row past q_lengths has zero weights and output.
+ *  - The dropout keeps w_ij, divided by 1 - drop_p, when u >= drop_p, and otherwise sets it
+ *    to 0. Here u = (fmix64(seed + fmix64(index)) >> 11) / 2^53, compared in double, where
+ *    fmix64 is the 64-bit finalizer of MurmurHash3 and index is the weight's row-major
+ *    position. drop_p must be in [0, 1), and 0 means no dropout.
+ *  - out = weights · v.
+ *  - The workspace holds only the status word (at least 256 bytes).
+ *  - Kernels. mma.sync tiles for bf16/fp16 with dqk = dv = 64 or 128. A SIMT kernel handles
+ *    the rest, or runs when SDPA_FLAG_GENERIC_KERNEL is set. */
+SDPA_API sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop_p, uint64_t seed, const void* q,
+                                               const void* k, const void* v, void* out, void* weights, void* ws,
+                                               size_t ws_bytes, struct CUstream_st* stream);
+
 /* Workspace bytes sdpa_backward needs for these params (256-byte aligned; 0 if invalid). */
 SDPA_API size_t sdpa_backward_workspace_size(const sdpa_params* p);
 
@@ -297,9 +317,10 @@ SDPA_API sdpa_status sdpa_read_device_status(void* ws, struct CUstream_st* strea
 /* Message for the last non-OK status returned on this host thread. */
 SDPA_API const char* sdpa_last_error(void);
 
-/* Name of the kernel the last sdpa_forward / sdpa_forward_packed / sdpa_decode_with_cache /
- * sdpa_backward call on this host thread launched for its attention ("generic_simt",
- * "prefill_tcgen05", "decode_splitkv", "backward_simt"). */
+/* Name of the kernel the last sdpa_forward / sdpa_forward_packed / sdpa_forward_with_weights /
+ * sdpa_decode_with_cache / sdpa_backward call on this host thread launched for its attention
+ * ("generic_simt", "prefill_tcgen05", "decode_splitkv", "weights_mma", "weights_simt",
+ * "backward_mma", "backward_simt"). */
 SDPA_API const char* sdpa_last_kernel(void);
 
 #ifdef __cplusplus

@@ -194,3 +194,16 @@ def test_backward_argument_rules():
     rc = sdpa.lib.sdpa_backward(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                                 need - 1, None)
     assert rc == sdpa.SDPA_ERR_WORKSPACE
+
+
+def test_with_weights_argument_rules():
+    """A drop probability outside [0, 1) and v_head_dim above 256 are rejected on the host."""
+    f = sdpa.lib.sdpa_forward_with_weights
+    for bad in (-0.1, 1.0, float("nan")):
+        p = _params()
+        assert f(ctypes.byref(p), bad, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == sdpa.SDPA_ERR_INVALID_ARG
+        assert "drop probability" in sdpa.lib.sdpa_last_error().decode()
+    p = _params(dv=320)
+    assert f(ctypes.byref(p), 0.0, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == sdpa.SDPA_ERR_UNSUPPORTED
+    p = _params()
+    assert f(ctypes.byref(p), 0.0, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1 << 20, None) == sdpa.SDPA_ERR_WORKSPACE
