@@ -56,3 +56,24 @@ def test_reproducible():
     b = si.qkv(si.TINY_FP32)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_packed_documents_recipe():
+    """Lengths in [seg_min, seg_max] (the last one cut to fit) adding up to the packed total;
+    the same seed gives the same documents."""
+    w = si.PACKED_DOCS
+    segs = si.packed_segments(w)
+    assert sum(segs) == w.q_len == w.kv_len
+    assert all(w.seg_min <= n <= w.seg_max for n in segs[:-1]) and 1 <= segs[-1] <= w.seg_max
+    assert segs == si.packed_segments(w) and len(segs) == 30
+    q, k, v = si.packed_qkv(si.scaled(w, q_len=100, kv_len=100))
+    assert q.shape == (100, 32, 128) and k.shape == v.shape == (100, 8, 128)
+
+
+def test_causal_pair_count():
+    """bench.causal_pairs (the flop count of every causal workload) against counting."""
+    import bench
+    for lq, lk, off in ((7, 7, 0), (5, 9, 4), (9, 5, -2), (1, 8192, 8191), (64, 64, -70)):
+        i = np.arange(lq)[:, None]
+        j = np.arange(lk)[None, :]
+        assert bench.causal_pairs(lq, lk, off) == int((j <= off + i).sum())
