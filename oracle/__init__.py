@@ -66,6 +66,9 @@ def load(path: str | None = None):
         lib = ctypes.CDLL(lib_path)
         lib.oracle_sdpa_forward.argtypes = [ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p]
         lib.oracle_sdpa_forward.restype = ctypes.c_int
+        lib.oracle_rope.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _i64p,
+                                    ctypes.c_double, _f64p]
+        lib.oracle_rope.restype = ctypes.c_int
         lib.oracle_sdpa_forward_with_weights.argtypes = [
             ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_uint64, _f64p, _f64p]
         lib.oracle_sdpa_forward_with_weights.restype = ctypes.c_int
@@ -185,6 +188,23 @@ def sdpa_forward(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_o
                                  _ptr(v, _f64p), _ptr(out, _f64p))
     if rc != 0:
         raise OracleError(f"oracle_sdpa_forward failed with code {rc}")
+    return out
+
+
+def rope(x, positions, base=10000.0, lib=None) -> np.ndarray:
+    """Rotary position embedding of x (..., nheads, d), positions one per row of the leading
+    dimensions: the pair (c, c + d/2) rotated by positions[t] * base^(-2c/d)."""
+    lib = lib or load()
+    x = _f64(x)
+    *lead, H, d = x.shape
+    rows = int(np.prod(lead)) if lead else 1
+    pos = np.ascontiguousarray(np.asarray(positions, dtype=np.int64).reshape(-1))
+    if pos.shape != (rows,):
+        raise ValueError(f"expected {rows} positions, got {pos.shape}")
+    out = np.empty_like(x)
+    rc = lib.oracle_rope(_ptr(x, _f64p), rows, H, d, _ptr(pos, _i64p), float(base), _ptr(out, _f64p))
+    if rc != 0:
+        raise OracleError(f"oracle_rope failed with code {rc}")
     return out
 
 

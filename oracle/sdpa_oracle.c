@@ -185,6 +185,33 @@ int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const dou
   return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
+/* Rotary position embedding of query or key rows (the Keras thread "MultiHeadAttention is
+ * missing a position_bias call argument": rotary embeddings applied to the key and query after
+ * the dense projections; the thread leaves the exact form open). Reading taken here, the common
+ * form: the head dimension d (even) is split in halves, and the pair (c, c + d/2),
+ * c < d/2, of row t is rotated by the angle positions[t] * base^(-2c/d):
+ *   out[c]       = x[c] cos a - x[c + d/2] sin a
+ *   out[c + d/2] = x[c + d/2] cos a + x[c] sin a
+ * x and out are [rows][nheads][d]; positions has one entry per row. */
+int oracle_rope(const double* x, int64_t rows, int64_t nheads, int64_t d, const int64_t* positions,
+                double base, double* out) {
+  if (!x || !out || !positions || rows < 0 || nheads <= 0 || d <= 0 || d % 2 || !(base > 0.0))
+    return ORACLE_ERR_ARG;
+  const int64_t half = d / 2;
+  for (int64_t t = 0; t < rows; ++t)
+    for (int64_t h = 0; h < nheads; ++h) {
+      const double* xr = x + (t * nheads + h) * d;
+      double* o = out + (t * nheads + h) * d;
+      for (int64_t c = 0; c < half; ++c) {
+        const double a = (double)positions[t] * pow(base, -2.0 * (double)c / (double)d);
+        const double x0 = xr[c], x1 = xr[c + half];
+        o[c] = x0 * cos(a) - x1 * sin(a);
+        o[c + half] = x1 * cos(a) + x0 * sin(a);
+      }
+    }
+  return ORACLE_OK;
+}
+
 /* Counter-based uniform draw for dropout: the 64-bit finalizer of Austin Appleby's MurmurHash3
  * ("fmix64"), applied twice, to the element's linear index (b, h, i, j) and then to that plus
  * the seed. The top 53 bits give u in [0, 1). */

@@ -382,6 +382,58 @@ def printed_example_shapes(lib):
         assert np.isfinite(out).all()
 
 
+# ---- rotary position embedding (the Keras thread's "rotary embeddings") ----------------------
+
+@pin
+def rope_two_dims_is_a_plane_rotation(lib):
+    """With d = 2 the single pair rotates by the position itself (frequency base^0 = 1):
+    the textbook plane rotation."""
+    x = _rng(91).standard_normal((5, 3, 2))
+    pos = np.array([0, 1, 7, -3, 1000])
+    out = oracle.rope(x, pos, lib=lib)
+    c, s_ = np.cos(pos)[:, None], np.sin(pos)[:, None]
+    _close(out[..., 0], x[..., 0] * c - x[..., 1] * s_)
+    _close(out[..., 1], x[..., 1] * c + x[..., 0] * s_)
+
+
+@pin
+def rope_is_a_rotation_by_relative_position(lib):
+    """Each pair is rotated, so norms are kept, position 0 is the identity, rotating by -p undoes
+    p, and q.k after the embedding depends only on the difference of the two positions (the
+    reason the embedding is applied to both query and key)."""
+    rng = _rng(92)
+    x = rng.standard_normal((6, 4, 64))
+    pos = rng.integers(-5000, 5000, size=6)
+    out = oracle.rope(x, pos, lib=lib)
+    _close(np.linalg.norm(out, axis=-1), np.linalg.norm(x, axis=-1))
+    _close(oracle.rope(x, np.zeros(6), lib=lib), x, 0.0)
+    _close(oracle.rope(out, -pos, lib=lib), x, 1e-11)
+    q, k = rng.standard_normal((2, 1, 2, 128))
+    for m, n, shift in ((3, 11, 100), (4000, 17, -2000), (0, 0, 12345)):
+        a = oracle.rope(q, [m], lib=lib)[0] @ oracle.rope(k, [n], lib=lib)[0].T
+        b = oracle.rope(q, [m + shift], lib=lib)[0] @ oracle.rope(k, [n + shift], lib=lib)[0].T
+        _close(a, b, 1e-9)
+
+
+@pin
+def rope_pairs_halves_with_geometric_frequencies(lib):
+    """A unit vector along dimension c < d/2 moves only within the plane of c and c + d/2, and
+    the angle measured at position 1 falls geometrically with c, from 1 radian, by the factor
+    base^(-2/d)."""
+    d, base = 16, 500.0
+    angles = []
+    for c in range(d // 2):
+        e = np.zeros((1, 1, d))
+        e[0, 0, c] = 1.0
+        out = oracle.rope(e, [1], base=base, lib=lib)[0, 0]
+        others = np.delete(out, [c, c + d // 2])
+        _close(others, np.zeros(d - 2), 0.0)
+        angles.append(math.atan2(out[c + d // 2], out[c]))
+    angles = np.array(angles)
+    _close(angles[0], 1.0, 1e-14)
+    _close(angles[1:] / angles[:-1], np.full(d // 2 - 1, base ** (-2 / d)), 1e-12)
+
+
 # ---- with weights and fdrop (the entry's "See also"; argument fdrop) -------------------------
 
 @pin

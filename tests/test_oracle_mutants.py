@@ -34,6 +34,9 @@ MUTANTS = {
     "block_class_swapped": ("(set == cells ? 2 : 1)", "(set == cells ? 1 : 2)"),
     "block_bits_reversed": ("word |= (1u << c);", "word |= (1u << (31 - c));"),
     "block_full_at_edge": ("(set == cells ? 2 : 1)", "(set == bq * bk ? 2 : 1)"),
+    "rope_pairs_adjacent": ("const double x0 = xr[c], x1 = xr[c + half];", "const double x0 = xr[c], x1 = xr[(c + 1) % d];"),
+    "rope_sin_sign": ("o[c] = x0 * cos(a) - x1 * sin(a);", "o[c] = x0 * cos(a) + x1 * sin(a);"),
+    "rope_frequency_exponent": ("pow(base, -2.0 * (double)c / (double)d)", "pow(base, -1.0 * (double)c / (double)d)"),
     "weights_dropout_unscaled": ("? w / (1.0 - drop_p) : 0.0", "? w : 0.0"),
     "weights_dropout_inverted": ("base + (uint64_t)j) >= drop_p)", "base + (uint64_t)j) < drop_p)"),
     "weights_head_batch_swapped": ("double* wrow = weights + ((b * H + h) * Lq + i) * Lk;",
