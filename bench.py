@@ -293,7 +293,8 @@ def other_workloads(args, dev, world, ws, peaks):
             ("block_sparse", "block_sparse_mask", lambda: block_sparse_workload(args, dev, world, ws, peaks)),
             ("packed", "packed_docs", lambda: packed_workload(args, dev, world, ws, peaks)),
             ("backward", "fused_gradient", lambda: backward_workload(args, dev, world, ws, peaks)),
-            ("weights", "with_weights", lambda: weights_workload(args, dev, world, ws, peaks)))
+            ("weights", "with_weights", lambda: weights_workload(args, dev, world, ws, peaks)),
+            ("rope", "rotary_embedding", lambda: rope_workload(args, dev, world, peaks)))
     res = {}
     for key, name, run in runs:
         if key not in args.workloads:
@@ -448,6 +449,31 @@ def weights_workload(args, dev, world, ws, peaks):
             "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 1}
 
 
+def rope_workload(args, dev, world, peaks):
+    """Rotary embedding of the causal GQA workload's q and k (positions 0..2047 in each
+    sequence): an elementwise pass, bound by reading and writing both arrays once."""
+    import head_scaled_dot_sdpa_b200 as sdpa
+
+    w = si.CAUSAL_GQA_PREFILL
+    q, k, _ = [t.to(dev) for t in si.qkv(w)]
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    pos = torch.arange(w.q_len, dtype=torch.int32, device=dev).repeat(w.batch)
+    byts = 2 * (q.numel() + k.numel()) * 2 + 2 * pos.numel() * 4
+
+    def step():
+        sdpa.sdpa_rope(q, pos, out=qo)
+        sdpa.sdpa_rope(k, pos, out=ko)
+
+    per = time_steps(step, args.steps, args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"workload": w.name + "_rope_qk", "metric": "HBM GB/s", "value": round(gbs * world, 1), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "bytes_per_step": byts,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm"], 4)},
+            "kernel": "rope_kernel", "gpu_launches_per_step": 2}
+
+
 # ---- CPU oracle ---------------------------------------------------------------------------------
 
 def _oracle_heads(q, k, v, heads, group):
@@ -528,7 +554,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--reference-heads", type=int, default=16)
-    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse,packed,backward,weights",
+    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse,packed,backward,weights,rope",
                     help="comma list; without 'prefill' only the other workloads run (a profiling aid)")
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide the decode batch and the block-sparse length by this (small ncu cases)")

@@ -80,6 +80,7 @@ _lib.sdpa_packed_workspace_size.restype = _sz
 _lib.sdpa_forward_packed.argtypes = [_PP, ctypes.POINTER(PackedSegments), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sdpa_forward_with_weights.argtypes = [_PP, ctypes.c_double, ctypes.c_uint64, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                            _vp]
+_lib.sdpa_rope.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int64, _i32, _i32, _vp, ctypes.c_double, _vp]
 _lib.sdpa_backward_workspace_size.argtypes = [_PP]
 _lib.sdpa_backward_workspace_size.restype = _sz
 _lib.sdpa_backward.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -94,7 +95,7 @@ _lib.sdpa_read_device_status.argtypes = [_vp, _vp]
 _lib.sdpa_last_error.restype = ctypes.c_char_p
 _lib.sdpa_last_kernel.restype = ctypes.c_char_p
 for _f in ("sdpa_workspace_init", "sdpa_forward", "sdpa_forward_packed", "sdpa_forward_with_weights",
-           "sdpa_backward", "sdpa_decode_with_cache",
+           "sdpa_rope", "sdpa_backward", "sdpa_decode_with_cache",
            "cache_update_at_index",
            "build_block_mask_info", "sdpa_read_device_status"):
     getattr(_lib, _f).restype = ctypes.c_int
@@ -299,6 +300,24 @@ def sdpa_forward_with_weights(q, k, v, bias=None, *, mask=None, scale=None, is_c
     return out, weights
 
 
+def sdpa_rope(x, positions, base=10000.0, *, out=None, stream=None):
+    """Rotary position embedding of x (..., nheads, d): the pair (c, c + d/2) of each row
+    rotated by positions[row] * base^(-2c/d), the rows being the leading dimensions flattened
+    (positions: one per row). out may be x."""
+    if not x.is_cuda or not x.is_contiguous() or x.dim() < 2 or x.dtype not in _DTYPE:
+        raise ValueError("x must be a contiguous float CUDA tensor (..., nheads, d)")
+    H, d = x.shape[-2], x.shape[-1]
+    rows = x.numel() // (H * d) if x.numel() else 0
+    pos = torch.as_tensor(positions, dtype=torch.int32, device=x.device).reshape(-1).contiguous()
+    if pos.numel() != rows:
+        raise ValueError(f"expected {rows} positions, got {pos.numel()}")
+    if out is None:
+        out = torch.empty_like(x)
+    _check(_lib.sdpa_rope(_ptr(x), _ptr(out), _DTYPE[x.dtype], rows, H, d, pos.data_ptr() if rows else None,
+                          float(base), _stream(stream)))
+    return out
+
+
 def sdpa_backward(q, k, v, out, dout, *, mask=None, scale=None, is_causal=False, q_offset=0,
                   q_lengths=None, kv_lengths=None, block_info=None, workspace=None, generic=False,
                   stream=None):
@@ -479,6 +498,6 @@ def build_block_mask_info(mask, bq: int = 128, bk: int = 128, *, stream=None) ->
     return info
 
 
-__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_forward_with_weights", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
+__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_forward_with_weights", "sdpa_rope", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
            "build_block_mask_info", "BlockMaskInfo", "Workspace", "read_device_status",
            "last_kernel", "SdpaError", "lib"]

@@ -99,6 +99,9 @@ cudaError_t launch_backward_mma(const Problem& P, const void* q, const void* k, 
 bool weights_mma_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out);
 cudaError_t launch_weights(const Problem& P, bool tiles, const void* q, const void* k, const void* v, void* out,
                            void* weights, double drop_p, unsigned long long seed, cudaStream_t stream);
+// Rotary position embedding of [rows][nheads][d] rows (out may alias x).
+cudaError_t launch_rope(int dtype, const void* x, void* out, long long rows, int nheads, int d,
+                        const int32_t* positions, double base, cudaStream_t stream);
 bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v,
                        const void* out);
 size_t prefill_workspace_bytes(const Problem& P);

@@ -286,6 +286,19 @@ sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop_p, uint6
   return SDPA_OK;
 }
 
+sdpa_status sdpa_rope(const void* x, void* out, sdpa_dtype dtype, int64_t rows, int32_t nheads, int32_t d,
+                      const int32_t* positions, double base, struct CUstream_st* stream) {
+  if (!valid_dtype(dtype)) return fail(SDPA_ERR_INVALID_ARG, "dtype is not an sdpa_dtype");
+  if (rows < 0 || nheads <= 0 || d <= 0 || d % 2 != 0)
+    return fail(SDPA_ERR_INVALID_ARG, "rotary embedding needs rows >= 0, nheads > 0 and an even head size (got %d)", d);
+  if (!(base > 0.0)) return fail(SDPA_ERR_INVALID_ARG, "rotary base must be positive");
+  if (rows == 0) return SDPA_OK;
+  if (!x || !out || !positions) return fail(SDPA_ERR_INVALID_ARG, "x, out and positions must not be NULL");
+  cudaError_t e = sdpa::launch_rope(dtype, x, out, rows, nheads, d, positions, base, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rotary embedding launch");
+  return SDPA_OK;
+}
+
 size_t sdpa_backward_workspace_size(const sdpa_params* p) {
   sdpa::Problem P;
   if (resolve(p, &P) != SDPA_OK) return 0;

@@ -219,6 +219,21 @@ SDPA_API sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop
                                                const void* k, const void* v, void* out, void* weights, void* ws,
                                                size_t ws_bytes, struct CUstream_st* stream);
 
+/* Rotary position embedding of query or key rows, applied after the projections and before
+ * attention (the Keras thread "MultiHeadAttention is missing a position_bias call argument"
+ * names rotary embeddings but gives no formula). The common form is used:
+ *    the pair (c, c + d/2), c < d/2, of row t is rotated by the angle a = positions[t] * base^(-2c/d):
+ *    out[c] = x[c] cos a - x[c + d/2] sin a,   out[c + d/2] = x[c + d/2] cos a + x[c] sin a.
+ *  - x, out: device arrays of `dtype`, [rows][nheads][d] (a padded batch flattens to
+ *    rows = batch * seq_len). out may be x (in place).
+ *  - positions: device int32[rows], the position of each row. With a KV cache this is the
+ *    absolute position, cache index + t.
+ *  - d must be even and base > 0 (10000 is the usual value). The angle and the rotation are
+ *    taken in double precision.
+ *  - One elementwise kernel; no workspace. */
+SDPA_API sdpa_status sdpa_rope(const void* x, void* out, sdpa_dtype dtype, int64_t rows, int32_t nheads, int32_t d,
+                               const int32_t* positions, double base, struct CUstream_st* stream);
+
 /* Workspace bytes sdpa_backward needs for these params (256-byte aligned; 0 if invalid). */
 SDPA_API size_t sdpa_backward_workspace_size(const sdpa_params* p);
 

@@ -207,3 +207,15 @@ def test_with_weights_argument_rules():
     assert f(ctypes.byref(p), 0.0, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == sdpa.SDPA_ERR_UNSUPPORTED
     p = _params()
     assert f(ctypes.byref(p), 0.0, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1 << 20, None) == sdpa.SDPA_ERR_WORKSPACE
+
+
+def test_rope_argument_rules():
+    """The rotary embedding needs an even head size, a positive base, and pointers when there
+    are rows; zero rows is a no-op."""
+    f = sdpa.lib.sdpa_rope
+    assert f(FAKE, FAKE, sdpa.SDPA_BF16, 4, 2, 63, FAKE, 10000.0, None) == sdpa.SDPA_ERR_INVALID_ARG
+    assert "even head size" in sdpa.lib.sdpa_last_error().decode()
+    assert f(FAKE, FAKE, sdpa.SDPA_BF16, 4, 2, 64, FAKE, 0.0, None) == sdpa.SDPA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 9, 4, 2, 64, FAKE, 10000.0, None) == sdpa.SDPA_ERR_INVALID_ARG
+    assert f(None, FAKE, sdpa.SDPA_BF16, 4, 2, 64, FAKE, 10000.0, None) == sdpa.SDPA_ERR_INVALID_ARG
+    assert f(None, None, sdpa.SDPA_BF16, 0, 2, 64, None, 10000.0, None) == sdpa.SDPA_OK
