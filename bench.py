@@ -53,36 +53,6 @@ def causal_pairs(Lq, Lk, offset=0):
     return int(np.clip(offset + i + 1, 0, Lk).sum())
 
 
-# ---- ncu figures committed under profiles/ ------------------------------------------------------
-
-PREFILL_SOURCES = ("prefill_sm100.cuh", "sm100_primitives.cuh", "prefill_sm100.cu")
-
-
-def source_hash(names):
-    """sha256 (first 16 hex digits) of the kernel's source files, in the given order."""
-    import hashlib
-    h = hashlib.sha256()
-    for n in names:
-        with open(os.path.join(ROOT, "head_scaled_dot_sdpa_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
-
-
-def profiled_traffic(summary, sources):
-    """DRAM bytes per launch recorded in a profiles/ summary, or None when the summary is
-    missing or was taken on other kernel sources than the current ones."""
-    import re
-    path = os.path.join(ROOT, "profiles", summary)
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    mh = re.search(r"source hash:\s*`?([0-9a-f]{16})", text)
-    mt = re.search(r"dram bytes per launch:\s*`?([0-9]+)", text)
-    if not mh or not mt or mh.group(1) != source_hash(sources):
-        return None
-    return int(mt.group(1))
-
-
 # ---- distributed plumbing -------------------------------------------------------------------
 
 def init_dist(n_gpus, backend=None):
@@ -244,8 +214,6 @@ def run_ours(args, rank, world, local):
     h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
     d2h = out.numel() * out.element_size()
 
-    traffic = profiled_traffic("prefill_tcgen05_causal_gqa_prefill.md", PREFILL_SOURCES)
-
     result.update({
         "metric": "prefill attention TFLOP/s (unmasked FLOPs)",
         "value": round(value, 2),
@@ -268,7 +236,7 @@ def run_ours(args, rank, world, local):
         "device_status": int(status),
         "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 2), "peak": peaks["bf16"],
                      "unit": "TFLOP/s", "frac": round(kernel_tflops / peaks["bf16"], 4),
-                     "traffic": traffic, "peak_source": f"{peaks['source']} bf16 burst",
+                     "traffic": None, "peak_source": f"{peaks['source']} bf16 burst",
                      "frac_of_sustained": round(kernel_tflops / peaks["bf16_sustained"], 4)},
         "e2e": {"value": round(flops * world / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
@@ -289,12 +257,13 @@ def other_workloads(args, dev, world, ws, peaks):
     """The other rows of the hot path, each timed like the headline. A workload that raises is
     reported as {"error": ...} so that the line with the headline is still printed."""
     runs = (("decode", "kv_cache_decode", lambda: decode_workload(args, dev, world, ws, peaks)),
-            ("bias", "alibi_t5_bias", lambda: bias_workload(args, dev, world, ws)),
+            ("bias", "alibi_t5_bias", lambda: bias_workload(args, dev, world, ws, peaks)),
             ("block_sparse", "block_sparse_mask", lambda: block_sparse_workload(args, dev, world, ws, peaks)),
             ("packed", "packed_docs", lambda: packed_workload(args, dev, world, ws, peaks)),
             ("backward", "fused_gradient", lambda: backward_workload(args, dev, world, ws, peaks)),
             ("weights", "with_weights", lambda: weights_workload(args, dev, world, ws, peaks)),
-            ("rope", "rotary_embedding", lambda: rope_workload(args, dev, world, peaks)))
+            ("rope", "rotary_embedding", lambda: rope_workload(args, dev, world, peaks)),
+            ("rope_prefill", "rope_prefill", lambda: rope_prefill_workload(args, dev, world, ws, peaks)))
     res = {}
     for key, name, run in runs:
         if key not in args.workloads:
@@ -332,22 +301,34 @@ def decode_workload(args, dev, world, ws, peaks):
             "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 4}
 
 
-def bias_workload(args, dev, world, ws):
-    """ALiBi/T5 bias attention (fp16, causal, additive bias)."""
+def bias_workload(args, dev, world, ws, peaks):
+    """ALiBi/T5 bias attention (fp16, causal, additive bias broadcast over the batch). Its
+    binding roof is HBM: the causal half of the bias (read once: both batch elements of a
+    (head, query tile) share it through L2) plus Q, K, V read and O written."""
     import head_scaled_dot_sdpa_b200 as sdpa
 
     w = si.ALIBI_T5_BIAS
     q, k, v = [t.to(dev) for t in si.qkv(w)]
     bias = si.alibi_t5_bias(w).to(dev)
     out = torch.empty_like(q)
-    flops = 4.0 * w.head_dim * w.batch * w.nheads * causal_pairs(w.q_len, w.kv_len)
+    pairs = causal_pairs(w.q_len, w.kv_len)
+    flops = 4.0 * w.head_dim * w.batch * w.nheads * pairs
     step = lambda: sdpa.sdpa_forward(q, k, v, bias, is_causal=True, out=out, workspace=ws)
     per = time_steps(step, args.steps, args.warmup, world)
     ms = max_over_ranks(float(np.mean(per)), world)
-    bias_bytes = w.nheads * causal_pairs(w.q_len, w.kv_len) * 2
-    return {"workload": w.name, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2),
-            "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
-            "bias_GBs": round(bias_bytes / (ms * 1e-3) / 1e9, 1), "kernel": sdpa.last_kernel()}
+    bias_bytes = w.nheads * pairs * 2
+    byts = bias_bytes + 4 * q.numel() * 2
+    gbs = byts / (ms * 1e-3) / 1e9
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "value": round(tf * world, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "flops_per_step": flops, "bytes_per_step": byts,
+            "bias_GBs": round(bias_bytes / (ms * 1e-3) / 1e9, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm"], 4), "traffic": None,
+                         "peak_source": f"{peaks['source']} HBM copy",
+                         "tensor": {"achieved": round(tf, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                                    "frac": round(tf / peaks["bf16"], 4)}},
+            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 1}
 
 
 def block_sparse_workload(args, dev, world, ws, peaks):
@@ -371,13 +352,24 @@ def block_sparse_workload(args, dev, world, ws, peaks):
     per = time_steps(step, args.steps, args.warmup, world)
     ms = max_over_ranks(float(np.mean(per)), world)
     flops = 4.0 * w.head_dim * allowed
-    n_blocks = int((cls != 0).sum())
+    # executed work: every (query, key) pair of the non-empty blocks (the diagonal forcing can
+    # turn an empty block partial, so the classes are counted from the classification itself)
+    n_blocks = int((info.arrays()["cls"] != 0).sum().item())
+    exec_flops = 4.0 * w.head_dim * n_blocks * 128 * 128
+    exec_tf = exec_flops / (ms * 1e-3) / 1e12
+    cgbs = mask.numel() / (ms_c * 1e-3) / 1e9
     return {
         "workload": w.name, "q_len": w.q_len, "value": round(flops / (ms * 1e-3) / 1e12 * world, 2), "unit": "TFLOP/s (unmasked)",
-        "ms_per_step": round(ms, 4), "executed_tflops": round(4.0 * w.head_dim * n_blocks * 128 * 128 / (ms * 1e-3) / 1e12, 2),
-        "classification": {"ms": round(ms_c, 4), "GB/s": round(mask.numel() / (ms_c * 1e-3) / 1e9, 1),
-                           "frac_hbm": round(mask.numel() / (ms_c * 1e-3) / 1e9 / peaks["hbm"], 4)},
-        "kernel": sdpa.last_kernel()}
+        "ms_per_step": round(ms, 4), "flops_per_step": flops, "executed_flops_per_step": exec_flops,
+        "executed_tflops": round(exec_tf, 2),
+        "roofline": {"bound": "tensor", "achieved": round(exec_tf, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": round(exec_tf / peaks["bf16"], 4), "traffic": None,
+                     "basis": "executed flops (non-empty 128x128 blocks)",
+                     "peak_source": f"{peaks['source']} bf16 burst"},
+        "classification": {"ms": round(ms_c, 4), "GB/s": round(cgbs, 1),
+                           "roofline": {"bound": "hbm", "achieved": round(cgbs, 1), "peak": peaks["hbm"],
+                                        "unit": "GB/s", "frac": round(cgbs / peaks["hbm"], 4)}},
+        "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 1}
 
 
 def packed_workload(args, dev, world, ws, peaks):
@@ -429,7 +421,9 @@ def backward_workload(args, dev, world, ws, peaks):
 def weights_workload(args, dev, world, ws, peaks):
     """scaled_dot_product_attention_with_weights with dropout (p = 0.1) on the causal GQA
     workload: the whole (batch, nheads, q_len, kv_len) weight array is written, so the step is
-    bound by that write (plus reading Q, K, V and writing out)."""
+    bound by that write (plus reading Q, K, V and writing out). The tcgen05 path runs three
+    kernels per step: the forward with the row log-sum-exp, the fill of the weights past each
+    query tile's causal bound, and the weights pass."""
     import head_scaled_dot_sdpa_b200 as sdpa
 
     w = si.CAUSAL_GQA_PREFILL
@@ -446,7 +440,8 @@ def weights_workload(args, dev, world, ws, peaks):
             "unit": "GB/s", "ms_per_step": round(ms, 3), "bytes_per_step": byts,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm"], 4)},
-            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 1}
+            "kernel": sdpa.last_kernel(),
+            "gpu_launches_per_step": 3 if sdpa.last_kernel() == "weights_tcgen05" else 1}
 
 
 def rope_workload(args, dev, world, peaks):
@@ -472,6 +467,29 @@ def rope_workload(args, dev, world, peaks):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm"], 4)},
             "kernel": "rope_kernel", "gpu_launches_per_step": 2}
+
+
+def rope_prefill_workload(args, dev, world, ws, peaks):
+    """The causal GQA prefill workload with the rotary embedding of q and k folded in
+    (sdpa_forward_rope, positions 0..2047 in every sequence): the keys are rotated once into the
+    workspace, a table kernel takes the query angles' cos / sin, and the attention kernel rotates
+    each Q tile in shared memory. TFLOP/s on the same flop count as the headline."""
+    import head_scaled_dot_sdpa_b200 as sdpa
+
+    w = si.CAUSAL_GQA_PREFILL
+    q, k, v = [t.to(dev) for t in si.qkv(w)]
+    out = torch.empty_like(q)
+    pos = torch.arange(w.q_len, dtype=torch.int32, device=dev).repeat(w.batch)
+    flops = 4.0 * w.head_dim * w.batch * w.nheads * causal_pairs(w.q_len, w.kv_len)
+    step = lambda: sdpa.sdpa_forward_rope(q, k, v, pos, pos, is_causal=True, out=out, workspace=ws)
+    per = time_steps(step, args.steps, args.warmup, world)
+    ms = max_over_ranks(float(np.mean(per)), world)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name + "_rope_fused", "value": round(tf * world, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16"], 4), "traffic": None},
+            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 3}
 
 
 # ---- CPU oracle ---------------------------------------------------------------------------------
@@ -554,7 +572,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--reference-heads", type=int, default=16)
-    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse,packed,backward,weights,rope",
+    ap.add_argument("--workloads", default="prefill,decode,bias,block_sparse,packed,backward,weights,rope,rope_prefill",
                     help="comma list; without 'prefill' only the other workloads run (a profiling aid)")
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide the decode batch and the block-sparse length by this (small ncu cases)")

@@ -9,7 +9,10 @@ Layout: q (B, Lq, H, dqk), k (B, Lk, Hkv, dqk), v (B, Lk, Hkv, dv), out (B, Lq, 
 row-major, i.e. the page's column-major (head_dim, nheads, seq_len, batch). A bias or mask is
 broadcastable to row-major (B, H, Lq, Lk), the page's (kv_len, q_len, nheads, batch).
 
-There is no fallback: if libsdpa.so is missing, importing this package raises.
+There is no fallback: if libsdpa.so is missing, importing this package raises. With
+SDPA_DEBUG_CHECKS=1 in the environment the package loads libsdpa_debug.so instead: the same
+kernels with every data-dependent device index range-checked (a violation is recorded as
+SDPA_ERR_DEVICE_CHECK in the status word instead of an out-of-range access).
 """
 from __future__ import annotations
 
@@ -20,11 +23,13 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsdpa.so")
+DEBUG_CHECKS = os.environ.get("SDPA_DEBUG_CHECKS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libsdpa_debug.so" if DEBUG_CHECKS else "libsdpa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing; build it with `python head_scaled_dot_sdpa_b200/build.py`")
+        f"{LIB_PATH} is missing; build it with `python head_scaled_dot_sdpa_b200/build.py"
+        f"{' --debug-checks' if DEBUG_CHECKS else ''}`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 # ---- ABI mirror -------------------------------------------------------------------------------
@@ -83,6 +88,11 @@ _lib.sdpa_forward_with_weights.argtypes = [_PP, ctypes.c_double, ctypes.c_uint64
 _lib.sdpa_rope.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int64, _i32, _i32, _vp, ctypes.c_double, _vp]
 _lib.sdpa_backward_workspace_size.argtypes = [_PP]
 _lib.sdpa_backward_workspace_size.restype = _sz
+_lib.sdpa_weights_workspace_size.argtypes = [_PP]
+_lib.sdpa_weights_workspace_size.restype = _sz
+_lib.sdpa_rope_workspace_size.argtypes = [_PP]
+_lib.sdpa_rope_workspace_size.restype = _sz
+_lib.sdpa_forward_rope.argtypes = [_PP, _vp, _vp, ctypes.c_double, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sdpa_backward.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sdpa_decode_with_cache.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.cache_update_at_index.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32,
@@ -276,6 +286,33 @@ def sdpa_forward(q, k, v, bias=None, *, mask=None, scale=None, is_causal=False, 
     return out
 
 
+def sdpa_forward_rope(q, k, v, q_positions, k_positions, bias=None, *, base=10000.0, mask=None, scale=None,
+                      is_causal=False, q_offset=0, q_lengths=None, kv_lengths=None, block_info=None, out=None,
+                      workspace=None, generic=False, stream=None):
+    """sdpa_forward on the rotary-embedded q and k (the pair (c, c + d/2) of each row rotated by
+    positions[row] * base^(-2c/d)), with q and k left as they are. q_positions: one per row of
+    q, (B, Lq) or B * Lq; k_positions: one per row of k."""
+    _check_qkv(q, k, v)
+    keep = []
+    p = _params(q, k, v, bias=bias, mask=mask, scale=scale, is_causal=is_causal, q_offset=q_offset,
+                q_lengths=q_lengths, kv_lengths=kv_lengths, block_info=block_info,
+                flags=SDPA_FLAG_GENERIC_KERNEL if generic else 0, keep=keep)
+    qp = torch.as_tensor(q_positions, dtype=torch.int32, device=q.device).reshape(-1).contiguous()
+    kp = torch.as_tensor(k_positions, dtype=torch.int32, device=q.device).reshape(-1).contiguous()
+    if qp.numel() != q.shape[0] * q.shape[1] or kp.numel() != k.shape[0] * k.shape[1]:
+        raise ValueError("one position per row of q and of k")
+    keep += [qp, kp]
+    if out is None:
+        out = torch.empty(q.shape[:3] + (v.shape[3],), dtype=q.dtype, device=q.device)
+    need = _lib.sdpa_rope_workspace_size(ctypes.byref(p))
+    if need == 0:
+        raise SdpaError(SDPA_ERR_INVALID_ARG, _lib.sdpa_last_error().decode())
+    ws = _workspace(q.device, need, workspace)
+    _check(_lib.sdpa_forward_rope(ctypes.byref(p), qp.data_ptr(), kp.data_ptr(), float(base), _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)))
+    return out
+
+
 def sdpa_forward_with_weights(q, k, v, bias=None, *, mask=None, scale=None, is_causal=False, q_offset=0,
                               q_lengths=None, kv_lengths=None, block_info=None, drop_p=0.0, seed=0, out=None,
                               weights=None, workspace=None, generic=False, stream=None):
@@ -293,7 +330,10 @@ def sdpa_forward_with_weights(q, k, v, bias=None, *, mask=None, scale=None, is_c
         out = torch.empty(q.shape[:3] + (v.shape[3],), dtype=q.dtype, device=q.device)
     if weights is None:
         weights = torch.empty((B, H, Lq, k.shape[1]), dtype=q.dtype, device=q.device)
-    ws = _workspace(q.device, 256, workspace)
+    need = _lib.sdpa_weights_workspace_size(ctypes.byref(p))
+    if need == 0:
+        raise SdpaError(SDPA_ERR_INVALID_ARG, _lib.sdpa_last_error().decode())
+    ws = _workspace(q.device, need, workspace)
     _check(_lib.sdpa_forward_with_weights(ctypes.byref(p), float(drop_p), int(seed) & (2**64 - 1), _ptr(q),
                                           _ptr(k), _ptr(v), _ptr(out), _ptr(weights), ws.ptr, ws.nbytes,
                                           _stream(stream)))
@@ -498,6 +538,6 @@ def build_block_mask_info(mask, bq: int = 128, bk: int = 128, *, stream=None) ->
     return info
 
 
-__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_forward_with_weights", "sdpa_rope", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
+__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_forward_rope", "sdpa_forward_with_weights", "sdpa_rope", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
            "build_block_mask_info", "BlockMaskInfo", "Workspace", "read_device_status",
            "last_kernel", "SdpaError", "lib"]

@@ -115,6 +115,8 @@ decode_split_kernel(Problem P, const T* __restrict__ q, const T* __restrict__ kc
   if (k0 >= kvlen) return;
   const int k1 = min(k0 + part.split, kvlen);
   const int R = n_new * gsz;  // rows r = t * gsz + hh
+  // range-checked build: keys inside the cache, the split inside the partials, rows in a tile
+  if (!SDPA_CHECKED(P.status, k1 <= cap && s < part.max_splits && R <= kRows)) return;
   const int off = kvlen - n_new;  // :bottom_right: query t attends keys j <= off + t
 
   const int grp = lane / 4, t4 = lane % 4;
@@ -328,10 +330,18 @@ __global__ void decode_combine_kernel(Problem P, Partials part, T* __restrict__ 
   const int t = (int)((row / P.H) % P.Lq);
   const int b = (int)(row / ((long long)P.H * P.Lq));
   const int idx = P.cache_index[b];
-  if (idx < 0 || idx > P.Lk - P.Lq) return;
+  T* orow = out + row * D;
+  if (idx < 0 || idx > P.Lk - P.Lq) {
+    // the sequence was skipped (reported by the cache update): NaN rows make that visible
+#pragma unroll
+    for (int u = 0; u < D / 32; ++u) orow[lane + 32 * u] = from_f32<T>(__int_as_float(0x7fc00000));
+    return;
+  }
   const int kvlen = idx + P.Lq;
-  const int n_splits = (kvlen + part.split - 1) / part.split;
+  int n_splits = (kvlen + part.split - 1) / part.split;
   const int kvh = h / P.group, r = t * P.group + (h % P.group);
+  // range-checked build: every split read lies inside the partials, every row inside a tile
+  if (!SDPA_CHECKED(P.status, n_splits <= part.max_splits && r < kRows)) n_splits = 0;
   const long long pbase = ((long long)b * P.Hkv + kvh) * part.max_splits;
   float M = -INFINITY;
   for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, part.ml[((pbase + s) * kRows + r) * 2]);
@@ -365,7 +375,6 @@ __global__ void decode_combine_kernel(Problem P, Partials part, T* __restrict__ 
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
   }
-  T* orow = out + row * D;
   const float inv = (L > 0.f) ? 1.f / L : __int_as_float(0x7fc00000);  // no key: NaN
 #pragma unroll
   for (int u = 0; u < kPer; ++u) orow[lane + 32 * u] = from_f32<T>(L > 0.f ? o[u] * inv : inv);

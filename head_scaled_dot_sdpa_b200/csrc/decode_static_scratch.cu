@@ -5,12 +5,14 @@
 // decode loop that must never block on (or fail in) the driver's allocator in the middle of a
 // run. They cannot provide the workspace sdpa_decode_with_cache needs for its split-KV
 // partials. sdpa_decode_with_cache_static gives them the same operation with the scratch in a
-// fixed-size array that lives in the library itself: SDPA_STATIC_SCRATCH_BYTES (32 MiB) of
+// fixed-size array that lives in the library itself: SDPA_STATIC_SCRATCH_BYTES (40 MiB) of
 // device memory, which every GPU that loads the library holds until the process exits.
 //
 // The array's name is only a host-side stand-in in host code, not a device address; its device
 // address is looked up once per device with cudaGetSymbolAddress, with that device current, and
-// then passed to the kernels. The first call on each device does that lookup.
+// then passed to the kernels. The first call on each device does that lookup. The first 256
+// bytes of the array are the status word area of the workspace layout; sdpa_read_static_status
+// reads and clears it.
 #include <cstdio>
 #include <mutex>
 
@@ -25,6 +27,33 @@ __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+
+// The array's device address on the current device (looked up on first use), or null with the
+// error message set.
+void* scratch_for_current_device(bool look_up, sdpa_status* st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    sdpa::set_last_error("cudaGetDevice failed or device ordinal out of range");
+    *st = SDPA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_scratch_ptr[dev] && look_up) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess || !ptr) {
+      char msg[256];
+      snprintf(msg, sizeof(msg), "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+      sdpa::set_last_error(msg);
+      *st = SDPA_ERR_CUDA;
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = ptr;
+  }
+  *st = SDPA_OK;
+  return g_scratch_ptr[dev];
+}
 
 }  // namespace
 
@@ -45,34 +74,19 @@ extern "C" sdpa_status sdpa_decode_with_cache_static(const sdpa_params* p, const
     sdpa::set_last_error(msg);
     return SDPA_ERR_WORKSPACE;
   }
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    sdpa::set_last_error("cudaGetDevice failed or device ordinal out of range");
-    return SDPA_ERR_CUDA;
-  }
-  void* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_ptr[dev]) {
-      void* ptr = nullptr;
-      e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-      if (e != cudaSuccess || !ptr) {
-        char msg[256];
-        snprintf(msg, sizeof(msg), "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
-        sdpa::set_last_error(msg);
-        return SDPA_ERR_CUDA;
-      }
-      g_scratch_ptr[dev] = ptr;
-    }
-    scratch = g_scratch_ptr[dev];
-  }
-  // the array keeps the previous call's contents: the status word must start at SDPA_OK
-  e = cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream);
-  if (e != cudaSuccess) {
-    sdpa::set_last_error("clearing the status word of the static scratch failed");
-    return SDPA_ERR_CUDA;
-  }
-  return sdpa_decode_with_cache(p, q, k_new, v_new, k_cache, v_cache, cache_index, out, scratch, kScratchBytes,
-                                stream);
+  sdpa_status st = SDPA_OK;
+  void* scratch = scratch_for_current_device(true, &st);
+  if (!scratch) return st;
+  // the array keeps the previous call's contents: the status word is cleared once the
+  // arguments have passed every check, before the kernels that may write it
+  return sdpa::decode_with_cache(p, q, k_new, v_new, k_cache, v_cache, cache_index, out, scratch, kScratchBytes,
+                                 (cudaStream_t)stream, true);
+}
+
+extern "C" sdpa_status sdpa_read_static_status(struct CUstream_st* stream) {
+  sdpa_status st = SDPA_OK;
+  void* scratch = scratch_for_current_device(false, &st);
+  if (st != SDPA_OK) return st;
+  if (!scratch) return SDPA_OK;  // no static call has run on this device
+  return sdpa_read_device_status(scratch, stream);
 }

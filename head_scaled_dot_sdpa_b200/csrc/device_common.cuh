@@ -26,6 +26,43 @@ __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, kStatusOk, code);
 }
 
+// Range checks of the build compiled with SDPA_DEBUG_CHECKS (libsdpa_debug.so): SDPA_CHECKED(st,
+// cond) is cond, and a false cond records SDPA_ERR_DEVICE_CHECK in the status word; the caller
+// then skips (or clamps) the access. In the normal build it is the constant true, and the
+// compiler removes the check.
+__device__ __forceinline__ bool checked(int* status, bool ok) {
+  if (!ok) report(status, SDPA_ERR_DEVICE_CHECK);
+  return ok;
+}
+#ifdef SDPA_DEBUG_CHECKS
+#define SDPA_CHECKED(status, cond) (::sdpa::checked((status), (cond)))
+#else
+#define SDPA_CHECKED(status, cond) (true)
+#endif
+
+// The dropout draw of scaled_dot_product_attention_with_weights (argument fdrop as dropout).
+// The weights' row-major positions (b, h, i, j) are taken four at a time: the group
+// index / 4 gets r = fmix64(seed + fmix64(index / 4)), fmix64 being the 64-bit finalizer of
+// Austin Appleby's MurmurHash3, and the weight at `index` takes 16-bit field index % 4 of r
+// (lowest first) as u in [0, 2^16); it is kept when u >= ceil(p * 2^16).
+__device__ __forceinline__ unsigned long long fmix64(unsigned long long k) {
+  k ^= k >> 33;
+  k *= 0xff51afd7ed558ccdULL;
+  k ^= k >> 33;
+  k *= 0xc4ceb9fe1a85ec53ULL;
+  k ^= k >> 33;
+  return k;
+}
+__device__ __forceinline__ unsigned long long dropout_group_draw(unsigned long long seed, unsigned long long group) {
+  return fmix64(seed + fmix64(group));
+}
+// bits f of the result: whether field f (f < 4) of r is kept
+__device__ __forceinline__ uint32_t dropout_keep4(unsigned long long r, unsigned threshold) {
+  return (uint32_t)(((unsigned)r & 0xFFFFu) >= threshold) | ((uint32_t)(((unsigned)(r >> 16) & 0xFFFFu) >= threshold) << 1) |
+         ((uint32_t)(((unsigned)(r >> 32) & 0xFFFFu) >= threshold) << 2) |
+         ((uint32_t)((unsigned)(r >> 48) >= threshold) << 3);
+}
+
 // Lengths, offsets: the arguments q_lengths, kv_lengths, q_offset and is_causal of
 // NNlib.scaled_dot_product_attention. Out-of-range lengths are clamped and reported.
 // With packed sequences (keywords q_segments / kv_segments, paragraph "Packed sequences") the

@@ -46,8 +46,14 @@ generic_attention_kernel(Problem P, const T* __restrict__ q, const T* __restrict
   // row (b, i, h) of a padded batch, or row i of packed sequence b (whose rows start at bi.q0;
   // rows past the sequence belong to the next one and are left alone)
   const BatchInfo bi = resolve_batch(P, b);
-  if (bi.skip || i >= bi.q_rows) return;
+  if (i >= bi.q_rows) return;
   const long long qi = (bi.q0 + i) * P.H + h;
+  if (bi.skip) {
+    // decode with an out-of-range cache index (reported by the cache update): NaN rows
+    T* orow = out + qi * Dv;
+    for (int e = lane; e < Dv; e += 32) orow[e] = from_f32<T>(__int_as_float(0x7fc00000));
+    return;
+  }
   float* qs = q_smem + warp * D;
   const T* qrow = q + qi * D;
   for (int c = lane; c < D; c += 32) qs[c] = to_f32(qrow[c]);

@@ -42,6 +42,18 @@ struct Problem {
   const int32_t* q_start;
   const int32_t* kv_start;
   int Lq_total, Lk_total;    // rows of the packed arrays
+  // scaled_dot_product_attention_with_weights on the tcgen05 kernel: the forward pass writes
+  // each row's log-sum-exp (log2 units, +inf for a row with no key or past q_lengths) to lse;
+  // the weights pass reads it, writes the weights [B][H][Lq][Lk] and applies the dropout
+  // (keep when the row's 16-bit draw >= drop_thr, then scale by inv_keep)
+  float* lse;
+  void* weights;
+  unsigned long long drop_seed;
+  unsigned drop_thr;
+  float inv_keep;
+  // rotary embedding of the Q tiles in shared memory (sdpa_forward_rope): cos / sin of each
+  // query row's angles, float2 [B * Lq][D / 2]; null when the queries are not rotated
+  const float2* q_rope;
   int* status;               // device status word (never null when a kernel runs)
   unsigned long long wait_timeout_ns;  // bound on every mbarrier wait of the tcgen05 kernel
   int selftest_stall;                  // SDPA_FLAG_SELFTEST_STALL
@@ -59,6 +71,13 @@ struct BatchInfo {
 
 // Records the message sdpa_last_error() returns on this host thread.
 void set_last_error(const char* msg);
+
+// sdpa_decode_with_cache. Every argument is checked before anything is queued; with
+// clear_status the status word at the start of `ws` is then zeroed on `stream` before the
+// kernels run (the allocation-free entry point, whose scratch keeps the previous call's bytes).
+sdpa_status decode_with_cache(const sdpa_params* p, const void* q, const void* k_new, const void* v_new,
+                              void* k_cache, void* v_cache, const int32_t* cache_index, void* out, void* ws,
+                              size_t ws_bytes, cudaStream_t stream, bool clear_status);
 
 // Launchers (each returns a cudaError_t from the launch).
 cudaError_t launch_generic(const Problem& P, const void* q, const void* k, const void* v,
@@ -102,8 +121,19 @@ cudaError_t launch_weights(const Problem& P, bool tiles, const void* q, const vo
 // Rotary position embedding of [rows][nheads][d] rows (out may alias x).
 cudaError_t launch_rope(int dtype, const void* x, void* out, long long rows, int nheads, int d,
                         const int32_t* positions, double base, cudaStream_t stream);
+// cos / sin of the rotary angles of `rows` positions: float2 table[rows][d / 2].
+cudaError_t launch_rope_table(long long rows, int d, const int32_t* positions, double base, void* table,
+                              cudaStream_t stream);
 bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v,
                        const void* out);
+// scaled_dot_product_attention_with_weights on the tcgen05 kernel (bf16 / fp16, head_dim =
+// v_head_dim = 64 or 128, no bias, mask or block info, kv_len a multiple of 8): the forward
+// with the row log-sum-exp into P.lse, the zero / NaN weights of the key tiles no query tile
+// visits, then the weights pass. P.lse, P.weights and the dropout fields must be set.
+bool prefill_weights_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out,
+                               const void* weights);
+cudaError_t launch_prefill_weights(const Problem& P, const void* q, const void* k, const void* v, void* out,
+                                   cudaStream_t stream, const char** error_message);
 size_t prefill_workspace_bytes(const Problem& P);
 cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const void* v,
                            void* out, void* ws_sched, cudaStream_t stream,

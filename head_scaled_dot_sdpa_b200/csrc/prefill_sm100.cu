@@ -103,6 +103,47 @@ bool prefill_supported(const Problem& P, const void* q, const void* k, const voi
 
 size_t prefill_workspace_bytes(const Problem&) { return 0; }
 
+bool prefill_weights_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out,
+                               const void* weights) {
+  return !P.bias && !P.mask && !P.bcls && !P.q_start && P.Lk % 8 == 0 && aligned(weights, 16) &&
+         prefill_supported(P, q, k, v, out);
+}
+
+cudaError_t launch_prefill_weights(const Problem& P, const void* q, const void* k, const void* v, void* out,
+                                   cudaStream_t stream, const char** msg) {
+  // 1. the forward, which also leaves each row's log-sum-exp in P.lse
+  cudaError_t e = launch_prefill(P, q, k, v, out, nullptr, stream, msg);
+  if (e != cudaSuccess) return e;
+  // 2. the weights of the key tiles the weights pass does not visit
+  const dim3 fgrid((unsigned)((P.Lq + prefill::kBlockM - 1) / prefill::kBlockM), (unsigned)P.H, (unsigned)P.B);
+  if (P.dtype == SDPA_BF16)
+    prefill::weights_fill_kernel<__nv_bfloat16><<<fgrid, 256, 0, stream>>>(P);
+  else
+    prefill::weights_fill_kernel<__half><<<fgrid, 256, 0, stream>>>(P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    if (msg) *msg = "weights fill launch";
+    return e;
+  }
+  // 3. the weights pass
+  prefill::TensorMaps maps{};
+  if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
+      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B)) {
+    if (msg) *msg = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
+  const int grid = (int)std::min<long long>(n_units, sm_count());
+  if (P.dtype == SDPA_BF16)
+    e = P.D == 128 ? prefill::launch_weights<__nv_bfloat16, 128>(maps, P, out, grid, stream)
+                   : prefill::launch_weights<__nv_bfloat16, 64>(maps, P, out, grid, stream);
+  else
+    e = P.D == 128 ? prefill::launch_weights<__half, 128>(maps, P, out, grid, stream)
+                   : prefill::launch_weights<__half, 64>(maps, P, out, grid, stream);
+  if (e != cudaSuccess && msg) *msg = "weights pass launch";
+  return e;
+}
+
 cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const void* v, void* out, void*,
                            cudaStream_t stream, const char** msg) {
   prefill::TensorMaps maps{};

@@ -63,8 +63,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 bytes (64 16-bit columns)
 constexpr int kNone = 1 << 30;
 constexpr int kUnitSlots = 4;        // ring of unit indices handed from the producer to the others
-constexpr int kUnitConsumers = 10;   // the two MMA warps and the 8 softmax warps
+constexpr int kUnitConsumers = 10;   // the two MMA warps and the 8 softmax warps (+ the rope warp)
 constexpr int kMmaWarpA = 9, kMmaWarpB = 11;  // MMA issuers of tile A and tile B
+constexpr int kRopeWarp = 10;        // rotates the Q tiles in shared memory when P.q_rope is set
 constexpr int kSchedWord = 16;       // int offset in the status area of the unit counter (+1: done)
 
 // bias / mask variants compiled into the kernel
@@ -72,23 +73,36 @@ constexpr int kSchedWord = 16;       // int offset in the status area of the uni
 // and key tile (head_dim 64, where the shared memory holds it); the others read global memory.
 enum { kBiasNone = 0, kBiasSame = 1, kBiasF32 = 2, kBiasTile = 3 };
 enum { kMaskNone = 0, kMaskDense = 1, kMaskBits = 2 };
+// kModeForward: the attention output (and, when P.lse is set, each row's log-sum-exp);
+// kModeWeights: scaled_dot_product_attention_with_weights given that log-sum-exp: the exact
+// weights 2^(x - lse) of the visited key tiles, dropped out and stored, and out = sum w' v.
+enum { kModeForward = 0, kModeWeights = 2 };
 
-template <int D>
+// Shared-memory plan. With bias tiles (kBT, head_dim 64) each query tile has kBiasSlots bias
+// tiles in flight, so the next key tile's bias streams in from HBM while the current one is
+// read; the K and V rings then keep 2 stages each to make room.
+template <int D, bool kBT = false>
 struct Cfg {
   static constexpr int kRegions = D / 64;
   static constexpr int kTileBytes = kRegions * kRegionBytes;
-  static constexpr int kKStages = D == 128 ? 2 : 4;
-  static constexpr int kVStages = D == 128 ? 2 : 4;
+  static constexpr int kKStages = (D == 128 || kBT) ? 2 : 4;
+  static constexpr int kVStages = (D == 128 || kBT) ? 2 : 4;
   static constexpr int kBiasTileBytes = 128 * 128 * 2;
-  static constexpr int kBarriers = 2 * 2 + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 + 1 + 2 * kUnitSlots;
-  // tiles (+ one bias tile per query tile), barriers, unit ring, TMEM address, abort flag, and
-  // slack to align the base to 1024 bytes
-  static constexpr int smem_bytes(bool bias_tiles) {
-    return (2 + kKStages + kVStages) * kTileBytes + (bias_tiles ? 2 * kBiasTileBytes : 0) + kBarriers * 8 + 64 +
-           1024;
+  static constexpr int kBiasSlots = 2;  // per query tile
+  // Q tiles: a ring shared by the two query tiles of the units, in the order A, B, A, B, ...
+  // With a third slot the next unit's tile A loads while the current unit still holds both.
+  static constexpr int kQSlots = kBT ? 2 : 3;
+  static constexpr int kBiasBytes = kBT ? 2 * kBiasSlots * kBiasTileBytes : 0;
+  static constexpr int kBarriers =
+      3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots;
+  // tiles (+ the bias tiles), barriers, unit ring, TMEM address, abort flag, and slack to align
+  // the base to 1024 bytes
+  static constexpr int smem_bytes() {
+    return (kQSlots + kKStages + kVStages) * kTileBytes + kBiasBytes + kBarriers * 8 + 64 + 1024;
   }
 };
-static_assert(Cfg<64>::smem_bytes(true) <= 227 * 1024, "bias tiles fit for head_dim 64");
+static_assert(Cfg<64, true>::smem_bytes() <= 227 * 1024, "bias tiles fit for head_dim 64");
+static_assert(Cfg<128>::smem_bytes() <= 227 * 1024 && Cfg<64>::smem_bytes() <= 227 * 1024, "tiles fit");
 
 struct TensorMaps {
   CUtensorMap q, k, v, bias;  // bias: (keys, queries, heads, batch), used by kBiasTile only
@@ -128,8 +142,11 @@ __device__ __forceinline__ QTile make_qtile(const Problem& P, const BatchInfo& b
   if (P.bcls) {
     const int hm = P.bi_nheads == 1 ? 0 : h;
     const long long row = (long long)hm * P.bi_nqb + qt;
+    // range-checked build: the block row must exist and its count fit the row
+    if (!SDPA_CHECKED(P.status, hm < P.bi_nheads && qt < P.bi_nqb)) return x;
     x.list = P.brow_list + row * P.bi_nkb;
-    const int cnt = P.brow_count[row];
+    int cnt = P.brow_count[row];
+    if (!SDPA_CHECKED(P.status, cnt >= 0 && cnt <= P.bi_nkb)) cnt = cnt < 0 ? 0 : P.bi_nkb;
     int n = 0;
     while (n < cnt && (int)(x.list[n] & 0x3FFFFFFFu) < n_lim) ++n;
     x.n = n;
@@ -230,21 +247,21 @@ __device__ __noinline__ void rescale_o(uint32_t taddr, float a) {
   tmem_wait_st();
 }
 
-template <typename T, int D, int kBias, int kMask>
+template <typename T, int D, int kBias, int kMask, int kMode = kModeForward>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __restrict__ out, int n_units) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kBias == kBiasTile>;
   using BT = typename std::conditional<kBias == kBiasF32, float, T>::type;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_smem = smem;  // [2] tiles
-  uint8_t* k_smem = q_smem + 2 * C::kTileBytes;
+  uint8_t* q_smem = smem;  // [kQSlots] tiles
+  uint8_t* k_smem = q_smem + C::kQSlots * C::kTileBytes;
   uint8_t* v_smem = k_smem + C::kKStages * C::kTileBytes;
-  uint8_t* b_smem = v_smem + C::kVStages * C::kTileBytes;  // [2] bias tiles (kBiasTile)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + (kBias == kBiasTile ? 2 * C::kBiasTileBytes : 0));
-  uint64_t* q_full = bars;                  // [2]
-  uint64_t* q_empty = q_full + 2;           // [2]
-  uint64_t* k_full = q_empty + 2;           // [KS]
+  uint8_t* b_smem = v_smem + C::kVStages * C::kTileBytes;  // [2][kBiasSlots] bias tiles (kBiasTile)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + C::kBiasBytes);
+  uint64_t* q_full = bars;                  // [kQSlots]
+  uint64_t* q_empty = q_full + C::kQSlots;  // [kQSlots]
+  uint64_t* k_full = q_empty + C::kQSlots;  // [KS]
   uint64_t* k_empty = k_full + C::kKStages;
   uint64_t* v_full = k_empty + C::kKStages; // [VS]
   uint64_t* v_empty = v_full + C::kVStages;
@@ -252,10 +269,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint64_t* p_full = s_full + 2;            // [2]
   uint64_t* o_ready = p_full + 2;           // [2]
   uint64_t* o_free = o_ready + 2;           // [2]
-  uint64_t* b_full = o_free + 2;            // [2] bias tile of the stream loaded
-  uint64_t* b_empty = b_full + 2;           // [2] bias tile read by the stream's softmax
-  uint64_t* drain = b_empty + 2;
-  uint64_t* unit_full = drain + 1;               // [kUnitSlots]
+  uint64_t* b_full = o_free + 2;            // [2][kBiasSlots] bias tile of the stream loaded
+  uint64_t* b_empty = b_full + 2 * C::kBiasSlots;  // [2][kBiasSlots] bias tile read by the stream's softmax
+  uint64_t* drain = b_empty + 2 * C::kBiasSlots;
+  uint64_t* q_rot = drain + 1;                   // [kQSlots] Q tile rotated (P.q_rope)
+  uint64_t* unit_full = q_rot + C::kQSlots;      // [kUnitSlots]
   uint64_t* unit_empty = unit_full + kUnitSlots; // [kUnitSlots]
   int* unit_ring = reinterpret_cast<int*>(unit_empty + kUnitSlots);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring + kUnitSlots);
@@ -267,15 +285,20 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   const uint64_t tmo = P.wait_timeout_ns;
 
   if (threadIdx.x == 0) {
+    for (int x = 0; x < C::kQSlots; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&q_rot[x], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4);  // one arrive per softmax warp
       mbar_init(&o_ready[s], 1);
       mbar_init(&o_free[s], 4);
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], kBlockM);
+    }
+    for (int x = 0; x < 2 * C::kBiasSlots; ++x) {
+      mbar_init(&b_full[x], 1);
+      mbar_init(&b_empty[x], 4);  // one arrive per softmax warp
     }
     // a K / V slot is released by both MMA warps
     for (int s = 0; s < C::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 2); }
@@ -283,7 +306,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     mbar_init(drain, 2);
     for (int k = 0; k < kUnitSlots; ++k) {
       mbar_init(&unit_full[k], 1);
-      mbar_init(&unit_empty[k], kUnitConsumers);
+      mbar_init(&unit_empty[k], kUnitConsumers + (P.q_rope ? 1 : 0));
     }
     *abort_flag = 0;
     issued[0] = 0;
@@ -339,8 +362,13 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     // ------------------------------------------------------------------ TMA producer
     [&] {
       uint32_t g = 0;            // key tiles loaded so far (ring position)
-      uint32_t qc[2] = {0, 0};   // Q tiles loaded per stream
+      uint32_t qi = 0;           // Q tiles loaded so far (ring position)
       uint32_t bc[2] = {0, 0};   // bias tiles loaded per stream
+      // extents of the tensor maps (packed sequences: one batch of all rows)
+      const bool packed_rows = P.q_start != nullptr;
+      const int q_rows_all = packed_rows ? P.Lq_total : P.Lq, kv_rows_all = packed_rows ? P.Lk_total : P.Lk;
+      const int n_batch = packed_rows ? 1 : P.B;
+      (void)q_rows_all; (void)kv_rows_all; (void)n_batch;
       // self-test: wait for a phase no one completes (the consumers' first release of slot 0)
       if (P.selftest_stall && !wait_all(&unit_empty[0], 0)) return;
       for (uint32_t k = 0;; ++k) {
@@ -370,14 +398,18 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           if (w.t[s].n == 0) continue;
-          if (!wait_all(&q_empty[s], (qc[s] & 1) ^ 1)) return;
+          const int qs = (int)(qi % C::kQSlots);
+          if (!wait_all(&q_empty[qs], ((qi / C::kQSlots) & 1) ^ 1)) return;
           if (elected) {
-            mbar_arrive_expect_tx(&q_full[s], C::kTileBytes);
+            int qh = w.t[s].h, qrow = w.tq + w.t[s].i0, qb = w.tb;
+            // range-checked build: a tile outside q is reported and read at the origin instead
+            if (!SDPA_CHECKED(P.status, qh < P.H && qrow < q_rows_all && qb < n_batch)) qh = qrow = qb = 0;
+            mbar_arrive_expect_tx(&q_full[qs], C::kTileBytes);
             for (int r = 0; r < C::kRegions; ++r)
-              tma_load_4d(q_smem + s * C::kTileBytes + r * kRegionBytes, &maps.q, &q_full[s], r * 64,
-                          w.t[s].h, w.tq + w.t[s].i0, w.tb);
+              tma_load_4d(q_smem + qs * C::kTileBytes + r * kRegionBytes, &maps.q, &q_full[qs], r * 64,
+                          qh, qrow, qb);
           }
-          ++qc[s];
+          ++qi;
         }
         // union of the two tiles' key lists; K_u is loaded ahead of V_{u-1}
         int ja = 0, jb = 0, prev_kb = -1;
@@ -389,10 +421,12 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             const int ks = x % C::kKStages;
             if (!wait_all(&k_empty[ks], ((x / C::kKStages) & 1) ^ 1)) return;
             if (elected) {
+              int kh = w.kvh, krow = w.tk + kb * kBlockN, kbt = w.tb;
+              if (!SDPA_CHECKED(P.status, kh < P.Hkv && krow < kv_rows_all && kbt < n_batch)) kh = krow = kbt = 0;
               mbar_arrive_expect_tx(&k_full[ks], C::kTileBytes);
               for (int r = 0; r < C::kRegions; ++r)
                 tma_load_4d(k_smem + ks * C::kTileBytes + r * kRegionBytes, &maps.k, &k_full[ks], r * 64,
-                            w.kvh, w.tk + kb * kBlockN, w.tb);
+                            kh, krow, kbt);
             }
           }
           if (prev_kb >= 0) {
@@ -400,26 +434,37 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             const int vs = x % C::kVStages;
             if (!wait_all(&v_empty[vs], ((x / C::kVStages) & 1) ^ 1)) return;
             if (elected) {
+              int vh = w.kvh, vrow = w.tk + prev_kb * kBlockN, vbt = w.tb;
+              if (!SDPA_CHECKED(P.status, vh < P.Hkv && vrow < kv_rows_all && vbt < n_batch)) vh = vrow = vbt = 0;
               mbar_arrive_expect_tx(&v_full[vs], C::kTileBytes);
               for (int r = 0; r < C::kRegions; ++r)
                 tma_load_4d(v_smem + vs * C::kTileBytes + r * kRegionBytes, &maps.v, &v_full[vs], r * 64,
-                            w.kvh, w.tk + prev_kb * kBlockN, w.tb);
+                            vh, vrow, vbt);
             }
           }
           if constexpr (kBias == kBiasTile) {
-            // the bias tile (queries of the stream's tile x keys of kb), once the stream's
-            // softmax has read the previous one; broadcast dimensions use coordinate 0
+            // the bias tile (queries of the stream's tile x keys of kb) into the stream's next
+            // slot, once the stream's softmax has read the tile that slot held; broadcast
+            // dimensions use coordinate 0. The stream's following bias tile is brought into L2
+            // now, one key tile ahead of its own load.
             if (kb != kNone) {
 #pragma unroll
               for (int s = 0; s < 2; ++s) {
                 if ((s == 0 ? na : nb) != kb) continue;
-                if (!wait_all(&b_empty[s], (bc[s] & 1) ^ 1)) return;
+                const int slot = (int)(bc[s] % C::kBiasSlots);
+                uint64_t* full = &b_full[s * C::kBiasSlots + slot];
+                if (!wait_all(&b_empty[s * C::kBiasSlots + slot], ((bc[s] / C::kBiasSlots) & 1) ^ 1)) return;
                 if (elected) {
-                  mbar_arrive_expect_tx(&b_full[s], C::kBiasTileBytes);
-                  const int hb = P.bs[2] != 0 ? w.t[s].h : 0, bb = P.bs[3] != 0 ? w.b : 0;
+                  int hb = P.bs[2] != 0 ? w.t[s].h : 0, bb = P.bs[3] != 0 ? w.b : 0;
+                  int bkey = kb * kBlockN, bq = w.t[s].i0;
+                  if (!SDPA_CHECKED(P.status, bkey < P.Lk && bq < P.Lq && hb < P.H && bb < P.B)) hb = bb = bkey = bq = 0;
+                  mbar_arrive_expect_tx(full, C::kBiasTileBytes);
+                  uint8_t* dst = b_smem + (s * C::kBiasSlots + slot) * C::kBiasTileBytes;
                   for (int r = 0; r < 2; ++r)
-                    tma_load_4d(b_smem + s * C::kBiasTileBytes + r * kRegionBytes, &maps.bias, &b_full[s],
-                                kb * kBlockN + r * 64, w.t[s].i0, hb, bb);
+                    tma_load_4d(dst + r * kRegionBytes, &maps.bias, full, bkey + r * 64, bq, hb, bb);
+                  const int kn = w.t[s].next((s == 0 ? ja : jb) + 1);
+                  if (kn != kNone && kn * kBlockN < P.Lk)
+                    for (int r = 0; r < 2; ++r) tma_prefetch_l2_4d(&maps.bias, kn * kBlockN + r * 64, bq, hb, bb);
                 }
                 ++bc[s];
               }
@@ -446,7 +491,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_qk = instr_desc_f16(kBf16, false, false, kBlockM, kBlockN);
       constexpr uint32_t idesc_pv = instr_desc_f16(kBf16, false, true, kBlockM, D);
-      const uint32_t qtile = smem_addr(q_smem) + s * C::kTileBytes;
+      const uint32_t q_base = smem_addr(q_smem);
       const uint32_t k_base = smem_addr(k_smem), v_base = smem_addr(v_smem);
       const uint32_t s_tmem = tmem + s * 128, o_tmem = tmem + 256 + s * D;
       // Turn order. A tile's MMAs come in groups: S(0); PV(j-1) + S(j); the last PV. Group k
@@ -474,7 +519,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       // the elected lane publishes a group as soon as its last MMA is issued (before the
       // commits): the other warp may then queue its own group behind it
       auto publish = [&]() { issued[s] = mine + 1; };
-      uint32_t g = 0, sc = 0, qc = 0, oc = 0;
+      uint32_t g = 0, sc = 0, qi = 0, oc = 0;  // qi: Q tiles of both streams so far (ring position)
       for (uint32_t kq = 0;; ++kq) {
         int u;
         if (!next_unit(kq, u)) return;
@@ -488,9 +533,14 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         const uint32_t groups_o = n_o > 0 ? (uint32_t)n_o + 1 : 0u;
         // group k of this tile may be issued once the other tile has issued `before(k)` groups
         auto before = [&](uint32_t k) -> uint32_t { return base_o + min(s == 0 ? k : k + 1, groups_o); };
+        // this tile's place in the Q ring: tile A, then tile B, of every unit with keys
+        const uint32_t my_qi = qi + ((s == 1 && w.t[0].n > 0) ? 1u : 0u);
+        qi += (w.t[0].n > 0 ? 1u : 0u) + (w.t[1].n > 0 ? 1u : 0u);
+        const int qslot = (int)(my_qi % C::kQSlots);
+        const uint32_t qtile = q_base + qslot * C::kTileBytes;
         if (my_n > 0) {
-          if (!wait_all(&q_full[s], qc & 1)) return;
-          ++qc;
+          // the Q tile loaded (and, with the rotary embedding, rotated in place)
+          if (!wait_all(P.q_rope ? &q_rot[qslot] : &q_full[qslot], (my_qi / C::kQSlots) & 1)) return;
         }
         // V(x) loaded and, for the unit's first PV, O free: waited for ahead of the turn, so
         // that they are off the path from "P ready" to the MMA issue
@@ -570,7 +620,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               mma_commit(&s_full[s]);
               mma_commit(&k_empty[ks]);
               // the tile's last S: Q may be reloaded once it completes
-              if (jm + 1 == my_n) mma_commit(&q_empty[s]);
+              if (jm + 1 == my_n) mma_commit(&q_empty[qslot]);
             }
             __syncwarp();
             ++mine;
@@ -599,6 +649,74 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         base_o += groups_o;
       }
     }();
+  } else if (warp == kRopeWarp) {
+    // ------------------------------------------------------------------ rotary embedding of Q
+    // Each Q tile, once loaded, is rotated in shared memory: the pair (c, c + D/2) of query row
+    // i by the angle whose cos / sin P.q_rope holds for row b * Lq + i. A lane takes 16-byte
+    // chunks (8 pairs) of one row; 128-byte swizzle: logical chunk x of row r is stored at
+    // chunk x ^ (r % 8). The writes are made visible to the tensor core (async proxy) before
+    // the tile is released to its MMA warp.
+    if (P.q_rope) [&] {
+      constexpr int kHalf = D / 2;
+      constexpr int kPairChunks = kHalf / 8;  // 16-byte chunk pairs per row
+      uint32_t qi = 0;
+      for (uint32_t kq = 0;; ++kq) {
+        int u;
+        if (!next_unit(kq, u)) return;
+        if (u >= n_units) break;
+        const Unit w = make_unit(P, u);
+        if (w.t[0].n == 0 && w.t[1].n == 0) continue;
+#pragma unroll 1
+        for (int s = 0; s < 2; ++s) {
+          const QTile qt = s ? w.t[1] : w.t[0];
+          if (qt.n == 0) continue;
+          const int qs = (int)(qi % C::kQSlots);
+          if (!wait_all(&q_full[qs], (qi / C::kQSlots) & 1)) return;
+          uint8_t* tile = q_smem + qs * C::kTileBytes;
+          const int rows = min(kBlockM, P.Lq - qt.i0);  // rows past the array are zeros
+#pragma unroll 1
+          for (int item = lane; item < rows * kPairChunks; item += 32) {
+            const int r = item / kPairChunks, x = item % kPairChunks;
+            // chunk x of the first half pairs with chunk x of the second half (D = 128: the
+            // second 64-column region; D = 64: chunk x + 4 of the one region)
+            uint8_t* lo = tile + r * 128 + ((x ^ (r & 7)) << 4);
+            uint8_t* hi = D == 128 ? lo + kRegionBytes : tile + r * 128 + (((x + 4) ^ (r & 7)) << 4);
+            const float4* cs = reinterpret_cast<const float4*>(
+                P.q_rope + ((long long)w.b * P.Lq + qt.i0 + r) * kHalf + 8 * x);
+            float tc[16];
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+              const float4 f = cs[z];
+              tc[4 * z] = f.x; tc[4 * z + 1] = f.y; tc[4 * z + 2] = f.z; tc[4 * z + 3] = f.w;
+            }
+            uint4 a = *reinterpret_cast<uint4*>(lo), b = *reinterpret_cast<uint4*>(hi);
+            uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
+            uint32_t* pb = reinterpret_cast<uint32_t*>(&b);
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+              float x0[2], x1[2];
+#pragma unroll
+              for (int y = 0; y < 2; ++y) {
+                const uint16_t la = (uint16_t)(pa[z] >> (16 * y)), lb = (uint16_t)(pb[z] >> (16 * y));
+                x0[y] = to_f32(*reinterpret_cast<const T*>(&la));
+                x1[y] = to_f32(*reinterpret_cast<const T*>(&lb));
+              }
+              const float c0 = tc[4 * z], s0 = tc[4 * z + 1], c1 = tc[4 * z + 2], s1 = tc[4 * z + 3];
+              const float y00 = x0[0] * c0 - x1[0] * s0, y10 = x1[0] * c0 + x0[0] * s0;
+              const float y01 = x0[1] * c1 - x1[1] * s1, y11 = x1[1] * c1 + x0[1] * s1;
+              pa[z] = std::is_same<T, __half>::value ? pack_f16x2(y00, y01) : pack_bf16x2(y00, y01);
+              pb[z] = std::is_same<T, __half>::value ? pack_f16x2(y10, y11) : pack_bf16x2(y10, y11);
+            }
+            *reinterpret_cast<uint4*>(lo) = a;
+            *reinterpret_cast<uint4*>(hi) = b;
+          }
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+          __syncwarp();
+          if (elected) mbar_arrive(&q_rot[qs]);
+          ++qi;
+        }
+      }
+    }();
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax + epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
@@ -618,9 +736,12 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if (qt.i0 == kNone) continue;  // the unit has no tile B
         const int i = qt.i0 + r;
         T* orow = out + ((w.o0 + i) * P.H + qt.h) * D;
+        // range-checked build: a row this thread would store must lie inside out
+        const bool row_ok = SDPA_CHECKED(P.status, i >= w.q_rows || (qt.h < P.H && w.o0 + i <
+                                         (P.q_start ? (long long)P.Lq_total : (long long)P.B * P.Lq)));
         if (qt.n == 0) {
           // no key tile: NaN rows (nothing attended) or zero rows (past q_lengths)
-          if (i < w.q_rows) {
+          if (i < w.q_rows && row_ok) {
             const float val = (i >= w.q_len) ? 0.f : __int_as_float(0x7fc00000);
             const uint32_t wv = std::is_same<T, __half>::value ? pack_f16x2(val, val) : pack_bf16x2(val, val);
 #pragma unroll
@@ -641,6 +762,20 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if constexpr (kMask == kMaskDense)
           mask_row = P.mask + (long long)i * P.ms[1] + (long long)qt.h * P.ms[2] + (long long)w.b * P.ms[3];
         float m_used = -INFINITY, l = 0.f;
+        // weights pass: the row's log-sum-exp from the forward (+inf: no key, or padding), the
+        // row of the weights, and its first position (the dropout counter)
+        float row_lse = INFINITY;
+        T* wrow = nullptr;
+        unsigned long long wbase = 0;
+        if constexpr (kMode == kModeWeights) {
+          const long long wr = ((long long)w.b * P.H + qt.h) * P.Lq + i;
+          if (i < P.Lq) {
+            row_lse = P.lse[wr];
+            wrow = static_cast<T*>(P.weights) + wr * P.Lk;
+            wbase = (unsigned long long)wr * (unsigned long long)P.Lk;
+          }
+          if (i < w.q_len && row_lse != INFINITY) l = 1.f;  // O is already normalised
+        }
         for (int j = 0; j < qt.n; ++j) {
           const int kb = qt.kb(j);
           const int key0 = kb * kBlockN;
@@ -650,8 +785,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if ((qt.list[j] >> 30) == SDPA_BLOCK_PARTIAL && nvalid > 0) {
               const int hm = P.bi_nheads == 1 ? 0 : qt.h;
               const long long blk = ((long long)hm * P.bi_nqb + qt.qt) * P.bi_nkb + kb;
-              const uint4 b4 = *reinterpret_cast<const uint4*>(P.bbits + (blk * kBlockM + r) * 4);
-              bw[0] = b4.x; bw[1] = b4.y; bw[2] = b4.z; bw[3] = b4.w;
+              // range-checked build: the block must lie inside the classification
+              if (SDPA_CHECKED(P.status, kb < P.bi_nkb && blk < (long long)P.bi_nheads * P.bi_nqb * P.bi_nkb)) {
+                const uint4 b4 = *reinterpret_cast<const uint4*>(P.bbits + (blk * kBlockM + r) * 4);
+                bw[0] = b4.x; bw[1] = b4.y; bw[2] = b4.z; bw[3] = b4.w;
+              }
             }
           }
           if (!wait_all(&s_full[s], sc & 1)) return;
@@ -661,6 +799,55 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + scol + c * 32, v[c]);
           tmem_wait_ld();
+          if constexpr (kMode == kModeWeights) {
+            // w = 2^(s * scale*log2e - lse) on the attended keys, 0 elsewhere, NaN for a row
+            // with no key; the dropout keeps w / (1 - p) where the row's draw allows; the
+            // weights go to global memory in 16-byte stores and w' into TMEM for the PV MMA
+            const bool nan_row = i < w.q_len && row_lse == INFINITY;
+            const float negl = nan_row ? 0.f : -row_lse;
+            const uint32_t nanw = std::is_same<T, __half>::value ? 0x7E007E00u : 0x7FC07FC0u;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int lim = nvalid - 32 * c;
+              uint32_t keep = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
+              if (P.drop_thr > 0) {
+                uint32_t kd = 0;
+                const unsigned long long g0 = (wbase + (unsigned long long)(key0 + 32 * c)) >> 2;
+#pragma unroll
+                for (int gq = 0; gq < 8; ++gq) kd |= dropout_keep4(dropout_group_draw(P.drop_seed, g0 + gq), P.drop_thr) << (4 * gq);
+                keep &= kd;
+              }
+              const float sc_keep = P.drop_thr > 0 ? P.inv_keep : 1.f;
+              uint32_t pk[16];
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float x0, x1;
+                fma2(x0, x1, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), sl2, sl2, negl, negl);
+                const float p0 = ((keep >> e) & 1u) ? ex2(x0) * sc_keep : 0.f;
+                const float p1 = ((keep >> (e + 1)) & 1u) ? ex2(x1) * sc_keep : 0.f;
+                pk[e / 2] = std::is_same<T, __half>::value ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+              }
+              if (wrow) {
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                  // 8 weights (kv_len is a multiple of 8, so a run is inside the row or past it)
+                  if (key0 + 32 * c + 2 * e < P.Lk) {
+                    const uint4 st = nan_row ? make_uint4(nanw, nanw, nanw, nanw) : make_uint4(pk[e], pk[e + 1], pk[e + 2], pk[e + 3]);
+                    *reinterpret_cast<uint4*>(wrow + key0 + 32 * c + 2 * e) = st;
+                  }
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[c / 2][(c % 2) * 16 + e] = pk[e];
+            }
+            tmem_st32(lane_addr + scol, v[0]);
+            tmem_st32(lane_addr + scol + 32, v[1]);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[s]);
+            continue;
+          }
           // Fast path (no bias, no mask bytes, every key of the tile attended by every row of
           // the warp): v keeps the raw scores, the max is taken on them (scale > 0) and the
           // exponent argument is one packed FMA, s * scale*log2e - m. Otherwise v becomes the
@@ -670,9 +857,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                                 (kMask == kMaskBits && (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu));
           const bool fast = kBias == kBiasNone && kMask != kMaskDense && __all_sync(0xffffffffu, full_row);
           float mul;
-          const uint8_t* bsm = b_smem + s * C::kBiasTileBytes;
+          const int bslot = s * C::kBiasSlots + (int)(bcs % C::kBiasSlots);
+          const uint8_t* bsm = b_smem + bslot * C::kBiasTileBytes;
           if constexpr (kBias == kBiasTile) {
-            if (!wait_all(&b_full[s], bcs & 1)) return;
+            if (!wait_all(&b_full[bslot], (bcs / C::kBiasSlots) & 1)) return;
           }
           if (kBias == kBiasNone && kMask != kMaskDense) {
             // No bias: the raw scores stay raw (the max commutes with scale > 0) and a masked
@@ -751,7 +939,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             }
           }
           if constexpr (kBias == kBiasTile) {
-            mbar_arrive(&b_empty[s]);  // the bias tile has been read
+            __syncwarp();  // every lane of the warp has read its bias row
+            if (lane == 0) mbar_arrive(&b_empty[bslot]);
             ++bcs;
           }
           const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * mul;
@@ -799,28 +988,36 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         tc_fence_after();
         const bool pad = i >= w.q_len;
         const float inv = (l > 0.f) ? 1.f / l : __int_as_float(0x7fc00000);
+        if constexpr (kMode == kModeForward) {
+          // the row's log-sum-exp in log2 units, for a weights pass that follows
+          if (P.lse && i < P.Lq)
+            P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = (!pad && l > 0.f) ? m_used + log2f(l) : INFINITY;
+        }
+        // O read out of TMEM in one batch (one wait), after which its columns are released to
+        // the next unit's first PV before the conversion and the stores
+        uint32_t o[D / 32][32];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + ocol + c * 32, o);
-          tmem_wait_ld();
-          if (i < w.q_rows) {
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_addr + ocol + c * 32, o[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[s]);
+        if (i < w.q_rows && row_ok) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint32_t wv[4];
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k]) * inv : inv);
-                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k + 1]) * inv : inv);
+                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[c][e + 2 * k]) * inv : inv);
+                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[c][e + 2 * k + 1]) * inv : inv);
                 wv[k] = std::is_same<T, __half>::value ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
               }
               *reinterpret_cast<uint4*>(orow + c * 32 + e) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free[s]);
       }
     }();
   }
@@ -858,10 +1055,44 @@ template <> cudaError_t launch<__nv_bfloat16, 64>(const TensorMaps&, const Probl
 template <> cudaError_t launch<__half, 128>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
 template <> cudaError_t launch<__half, 64>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
 
-template <typename T, int D, int kBias, int kMask>
+// The weights pass (kModeWeights, no bias or mask) for one (T, D) pair, after the forward has
+// written P.lse and weights_fill_kernel the key tiles the pass does not visit.
+template <typename T, int D>
+cudaError_t launch_weights(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream);
+template <> cudaError_t launch_weights<__nv_bfloat16, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_weights<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_weights<__half, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_weights<__half, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+
+// The weights of the key tiles a query tile does not visit (past its causal / kv_lengths bound,
+// the tiles make_qtile leaves out): 0, or NaN for a row with no key. Grid (query tiles, H, B);
+// kv_len is a multiple of 8, so each row's run starts on a 16-byte boundary.
+template <typename T>
+__global__ void __launch_bounds__(256) weights_fill_kernel(const Problem P) {
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const BatchInfo bi = resolve_batch(P, b);
+  const QTile x = make_qtile(P, bi, h, qt, true);
+  const int col0 = x.n * kBlockN;
+  if (col0 >= P.Lk) return;
+  const int chunks = (P.Lk - col0) / 8;  // 16-byte runs per row
+  const int rows = min(kBlockM, P.Lq - qt * kBlockM);
+  const uint32_t nanw = std::is_same<T, __half>::value ? 0x7E007E00u : 0x7FC07FC0u;
+  T* base = static_cast<T*>(P.weights);
+  for (int idx = threadIdx.x; idx < rows * chunks; idx += blockDim.x) {
+    const int r = idx / chunks, c = idx % chunks;
+    const int i = qt * kBlockM + r;
+    long long lim = (i < bi.q_len) ? bi.kv_len : 0;
+    if (P.causal != SDPA_CAUSAL_NONE) lim = min(lim, (long long)bi.offset + i + 1);
+    const bool nan_row = i < bi.q_len && lim <= 0;
+    T* row = base + (((long long)b * P.H + h) * P.Lq + i) * P.Lk + col0;
+    reinterpret_cast<uint4*>(row)[c] = nan_row ? make_uint4(nanw, nanw, nanw, nanw) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <typename T, int D, int kBias, int kMask, int kMode = kModeForward>
 cudaError_t launch_variant(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream) {
-  auto kern = prefill_kernel<T, D, kBias, kMask>;
-  const int smem = Cfg<D>::smem_bytes(kBias == kBiasTile);
+  auto kern = prefill_kernel<T, D, kBias, kMask, kMode>;
+  const int smem = Cfg<D, kBias == kBiasTile>::smem_bytes();
   // checked and configured once per device (bit d of `ready`)
   static std::atomic<unsigned long long> ready{0};
   int dev = 0;
@@ -895,6 +1126,11 @@ inline int mask_variant(const Problem& P) {
 }
 
 #define SDPA_PREFILL_DEFINE_LAUNCH(T, D)                                                              \
+  template <>                                                                                       \
+  cudaError_t launch_weights<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,  \
+                                   cudaStream_t stream) {                                           \
+    return launch_variant<T, D, kBiasNone, kMaskNone, kModeWeights>(maps, P, out, grid, stream);   \
+  }                                                                                                 \
   template <>                                                                                       \
   cudaError_t launch<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,         \
                            bool bias_tiles, cudaStream_t stream) {                                  \

@@ -3,51 +3,145 @@
 // applied to the key and query). The form used: the pair (c, c + d/2) of row t is rotated by
 // the angle positions[t] * base^(-2c/d).
 //
-// An HBM-bound elementwise pass: one thread per pair, consecutive threads on consecutive c of a
-// row, so both halves are read and written in coalesced runs. The angle, its sine and cosine
-// and the rotation are taken in double precision, so fp32 rows keep full accuracy at positions
-// of 10^5 and more. Each pair is read before it is written by the same thread, so out may
-// alias x.
+// An HBM-bound elementwise pass. The angle of (row t, pair c) is the same for every head, so one
+// thread takes VEC consecutive pairs of one row, computes their sines and cosines once and
+// rotates those pairs in all nheads heads; the threads of a warp cover consecutive pairs, so
+// each head's two halves are read and written in coalesced runs (VEC = 2: 4-byte 16-bit pairs).
+// The frequencies base^(-2c/d) are a per-block table in double precision. The angle is formed
+// and reduced to [-pi, pi] in double precision (positions of 10^5 and more keep their accuracy),
+// then CUDA's sincosf evaluates it in single precision. Each element is read before it is
+// written by the same thread, so out may alias x.
 #include "device_common.cuh"
 
 namespace sdpa {
 namespace {
 
-template <typename T>
-__global__ void __launch_bounds__(256)
+constexpr int kThreads = 256;
+
+template <typename T, int VEC>
+__global__ void __launch_bounds__(kThreads)
 rope_kernel(const T* x, T* out, long long rows, int nheads, int d, const int32_t* __restrict__ positions,
             double log2_base) {
+  extern __shared__ double freq[];  // [d / 2]
   const int half = d / 2;
-  const long long pairs = rows * nheads * half;
-  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < pairs;
+  for (int c = threadIdx.x; c < half; c += blockDim.x) freq[c] = exp2(-2.0 * (double)c / (double)d * log2_base);
+  __syncthreads();
+  const int groups = half / VEC;  // pair groups per row
+  const long long items = rows * groups;
+  const long long row_elems = (long long)nheads * d;
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < items;
        idx += (long long)gridDim.x * blockDim.x) {
-    const int c = (int)(idx % half);
-    const long long rh = idx / half;  // (row, head)
-    const long long t = rh / nheads;
-    const double a = (double)positions[t] * exp2(-2.0 * (double)c / (double)d * log2_base);
-    double sn, cs;
-    sincos(a, &sn, &cs);
-    const double x0 = to_f32(x[rh * d + c]), x1 = to_f32(x[rh * d + c + half]);
-    out[rh * d + c] = from_f32<T>((float)(x0 * cs - x1 * sn));
-    out[rh * d + c + half] = from_f32<T>((float)(x1 * cs + x0 * sn));
+    const long long t = idx / groups;
+    const int c0 = (int)(idx % groups) * VEC;
+    const double pos = (double)positions[t];
+    float cs[VEC], sn[VEC];
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) {
+      const double a = pos * freq[c0 + u];
+      const double r = a - kTwoPi * rint(a / kTwoPi);  // in [-pi, pi]
+      sincosf((float)r, &sn[u], &cs[u]);
+    }
+    const T* xr = x + t * row_elems + c0;
+    T* orow = out + t * row_elems + c0;
+    for (int h = 0; h < nheads; ++h) {
+      float x0[VEC], x1[VEC];
+      if constexpr (VEC == 2 && sizeof(T) == 2) {
+        const uint32_t a = *reinterpret_cast<const uint32_t*>(xr + (long long)h * d);
+        const uint32_t b = *reinterpret_cast<const uint32_t*>(xr + (long long)h * d + half);
+        const T* pa = reinterpret_cast<const T*>(&a);
+        const T* pb = reinterpret_cast<const T*>(&b);
+        x0[0] = to_f32(pa[0]); x0[1] = to_f32(pa[1]);
+        x1[0] = to_f32(pb[0]); x1[1] = to_f32(pb[1]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) {
+          x0[u] = to_f32(xr[(long long)h * d + u]);
+          x1[u] = to_f32(xr[(long long)h * d + half + u]);
+        }
+      }
+      T y0[VEC], y1[VEC];
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) {
+        y0[u] = from_f32<T>(x0[u] * cs[u] - x1[u] * sn[u]);
+        y1[u] = from_f32<T>(x1[u] * cs[u] + x0[u] * sn[u]);
+      }
+      if constexpr (VEC == 2 && sizeof(T) == 2) {
+        *reinterpret_cast<uint32_t*>(orow + (long long)h * d) = *reinterpret_cast<const uint32_t*>(y0);
+        *reinterpret_cast<uint32_t*>(orow + (long long)h * d + half) = *reinterpret_cast<const uint32_t*>(y1);
+      } else {
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) {
+          orow[(long long)h * d + u] = y0[u];
+          orow[(long long)h * d + half + u] = y1[u];
+        }
+      }
+    }
   }
 }
 
 template <typename T>
 cudaError_t launch_t(const void* x, void* out, long long rows, int nheads, int d, const int32_t* positions,
                      double base, cudaStream_t stream) {
-  const long long pairs = rows * nheads * (d / 2);
-  if (pairs == 0) return cudaSuccess;
+  const int half = d / 2;
+  if (rows == 0 || half == 0) return cudaSuccess;
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long blocks = (pairs + 255) / 256;
-  const unsigned grid = (unsigned)(blocks < 16LL * sms ? blocks : 16LL * sms);
-  rope_kernel<T><<<grid, 256, 0, stream>>>((const T*)x, (T*)out, rows, nheads, d, positions, log2(base));
+  // 16-bit pairs of two consecutive c: both halves of every row start on a 4-byte boundary when
+  // half is even and the arrays are 4-byte aligned
+  const bool vec2 = sizeof(T) == 2 && half % 2 == 0 && (reinterpret_cast<uintptr_t>(x) % 4 == 0) &&
+                    (reinterpret_cast<uintptr_t>(out) % 4 == 0);
+  const long long items = rows * (vec2 ? half / 2 : half);
+  const long long blocks = (items + kThreads - 1) / kThreads;
+  const unsigned grid = (unsigned)(blocks < 8LL * sms ? blocks : 8LL * sms);
+  const size_t smem = sizeof(double) * half;
+  if (vec2)
+    rope_kernel<T, 2><<<grid, kThreads, smem, stream>>>((const T*)x, (T*)out, rows, nheads, d, positions, log2(base));
+  else
+    rope_kernel<T, 1><<<grid, kThreads, smem, stream>>>((const T*)x, (T*)out, rows, nheads, d, positions, log2(base));
   return cudaGetLastError();
 }
 
+// cos / sin of every (row, pair c) angle, interleaved: table[(row * (d/2) + c) * 2 + {0, 1}],
+// the angle formed and reduced as in rope_kernel. The prefill kernel reads it to rotate its Q
+// tiles in shared memory.
+__global__ void __launch_bounds__(kThreads)
+rope_table_kernel(long long rows, int d, const int32_t* __restrict__ positions, double log2_base,
+                  float2* __restrict__ table) {
+  extern __shared__ double freq[];  // [d / 2]
+  const int half = d / 2;
+  for (int c = threadIdx.x; c < half; c += blockDim.x) freq[c] = exp2(-2.0 * (double)c / (double)d * log2_base);
+  __syncthreads();
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  const long long items = rows * half;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < items;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long t = idx / half;
+    const int c = (int)(idx % half);
+    const double a = (double)positions[t] * freq[c];
+    const double r = a - kTwoPi * rint(a / kTwoPi);
+    float sn, cs;
+    sincosf((float)r, &sn, &cs);
+    table[idx] = make_float2(cs, sn);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_rope_table(long long rows, int d, const int32_t* positions, double base, void* table,
+                              cudaStream_t stream) {
+  const int half = d / 2;
+  if (rows == 0 || half == 0) return cudaSuccess;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long blocks = (rows * half + kThreads - 1) / kThreads;
+  const unsigned grid = (unsigned)(blocks < 8LL * sms ? blocks : 8LL * sms);
+  rope_table_kernel<<<grid, kThreads, sizeof(double) * half, stream>>>(rows, d, positions, log2(base),
+                                                                       static_cast<float2*>(table));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rope(int dtype, const void* x, void* out, long long rows, int nheads, int d,
                         const int32_t* positions, double base, cudaStream_t stream) {

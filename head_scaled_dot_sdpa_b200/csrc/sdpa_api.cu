@@ -263,6 +263,12 @@ sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed_segments
   return SDPA_OK;
 }
 
+size_t sdpa_weights_workspace_size(const sdpa_params* p) {
+  sdpa::Problem P;
+  if (resolve(p, &P) != SDPA_OK) return 0;
+  return kStatusBytes + round256((size_t)P.B * P.H * P.Lq * sizeof(float));
+}
+
 sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop_p, uint64_t seed, const void* q,
                                       const void* k, const void* v, void* out, void* weights, void* ws,
                                       size_t ws_bytes, struct CUstream_st* stream) {
@@ -272,12 +278,27 @@ sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop_p, uint6
   if (!(drop_p >= 0.0 && drop_p < 1.0)) return fail(SDPA_ERR_INVALID_ARG, "drop probability %g is not in [0, 1)", drop_p);
   if (P.Dv > 256) return fail(SDPA_ERR_UNSUPPORTED, "v_head_dim %d exceeds the weights kernels' limit (256)", P.Dv);
   if (P.D > 1024) return fail(SDPA_ERR_UNSUPPORTED, "head_dim %d exceeds the weights kernels' limit (1024)", P.D);
-  st = check_workspace(ws, ws_bytes, kStatusBytes);
+  st = check_workspace(ws, ws_bytes, sdpa_weights_workspace_size(p));
   if (st != SDPA_OK) return st;
   if ((long long)P.B * P.Lq * P.H == 0) return SDPA_OK;
   if (!q || !out || !weights || (P.Lk > 0 && (!k || !v)))
     return fail(SDPA_ERR_INVALID_ARG, "q, k, v, out and weights must not be NULL");
   P.status = static_cast<int*>(ws);
+  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && P.Lk > 0 &&
+      sdpa::prefill_weights_supported(P, q, k, v, out, weights)) {
+    // tcgen05: the forward (with the row log-sum-exp in the workspace), the weights of the
+    // unvisited key tiles, then the weights pass
+    P.lse = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
+    P.weights = weights;
+    P.drop_seed = (unsigned long long)seed;
+    P.drop_thr = drop_p > 0.0 ? (unsigned)std::ceil(drop_p * 65536.0) : 0u;
+    P.inv_keep = (float)(1.0 / (1.0 - drop_p));
+    const char* msg = nullptr;
+    cudaError_t e = sdpa::launch_prefill_weights(P, q, k, v, out, (cudaStream_t)stream, &msg);
+    if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "weights launch");
+    g_last_kernel = "weights_tcgen05";
+    return SDPA_OK;
+  }
   const bool tiles = !(p->flags & SDPA_FLAG_GENERIC_KERNEL) && P.Lk > 0 && sdpa::weights_mma_supported(P, q, k, v, out);
   cudaError_t e = sdpa::launch_weights(P, tiles, q, k, v, out, weights, drop_p, (unsigned long long)seed,
                                        (cudaStream_t)stream);
@@ -292,10 +313,82 @@ sdpa_status sdpa_rope(const void* x, void* out, sdpa_dtype dtype, int64_t rows, 
   if (rows < 0 || nheads <= 0 || d <= 0 || d % 2 != 0)
     return fail(SDPA_ERR_INVALID_ARG, "rotary embedding needs rows >= 0, nheads > 0 and an even head size (got %d)", d);
   if (!(base > 0.0)) return fail(SDPA_ERR_INVALID_ARG, "rotary base must be positive");
+  if (d > 8192) return fail(SDPA_ERR_UNSUPPORTED, "rotary embedding supports head sizes up to 8192 (got %d)", d);
   if (rows == 0) return SDPA_OK;
   if (!x || !out || !positions) return fail(SDPA_ERR_INVALID_ARG, "x, out and positions must not be NULL");
   cudaError_t e = sdpa::launch_rope(dtype, x, out, rows, nheads, d, positions, base, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "rotary embedding launch");
+  return SDPA_OK;
+}
+
+// Workspace of sdpa_forward_rope: the status word, then the rotated keys, the cos / sin table
+// of the query rows (the tcgen05 kernel rotates its Q tiles with it) and room for rotated
+// queries (the other kernels take them from memory).
+namespace {
+struct RopeLayout {
+  size_t k_off, table_off, q_off, total;
+};
+RopeLayout rope_layout(const sdpa::Problem& P) {
+  RopeLayout L;
+  const size_t es = P.dtype == SDPA_F32 ? 4 : 2;
+  L.k_off = kStatusBytes;
+  L.table_off = L.k_off + round256((size_t)P.B * P.Lk * P.Hkv * P.D * es);
+  L.q_off = L.table_off + round256((size_t)P.B * P.Lq * (P.D / 2) * 2 * sizeof(float));
+  L.total = L.q_off + round256((size_t)P.B * P.Lq * P.H * P.D * es) +
+            round256(sdpa::prefill_workspace_bytes(P));
+  return L;
+}
+}  // namespace
+
+size_t sdpa_rope_workspace_size(const sdpa_params* p) {
+  sdpa::Problem P;
+  if (resolve(p, &P) != SDPA_OK || P.D % 2 != 0) return 0;
+  return rope_layout(P).total;
+}
+
+sdpa_status sdpa_forward_rope(const sdpa_params* p, const int32_t* q_positions, const int32_t* k_positions,
+                              double base, const void* q, const void* k, const void* v, void* out, void* ws,
+                              size_t ws_bytes, struct CUstream_st* stream) {
+  sdpa::Problem P;
+  sdpa_status st = resolve(p, &P);
+  if (st != SDPA_OK) return st;
+  if (P.D % 2 != 0 || P.D > 8192)
+    return fail(SDPA_ERR_INVALID_ARG, "the rotary embedding needs an even qk_head_dim of at most 8192 (got %d)", P.D);
+  if (!(base > 0.0)) return fail(SDPA_ERR_INVALID_ARG, "rotary base must be positive");
+  const RopeLayout L = rope_layout(P);
+  st = check_workspace(ws, ws_bytes, L.total);
+  if (st != SDPA_OK) return st;
+  if ((long long)P.B * P.Lq * P.H == 0) return SDPA_OK;
+  if (!q || !out || (P.Lk > 0 && (!k || !v || !k_positions)) || !q_positions)
+    return fail(SDPA_ERR_INVALID_ARG, "q, k, v, out and the positions must not be NULL");
+  P.status = static_cast<int*>(ws);
+  char* base_ws = static_cast<char*>(ws);
+  void* k_rot = base_ws + L.k_off;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the keys, rotated once: every query tile of the key/value head reads them
+  cudaError_t e = sdpa::launch_rope(P.dtype, k, k_rot, (long long)P.B * P.Lk, P.Hkv, P.D, k_positions, base, s);
+  if (e != cudaSuccess) return cuda_fail(e, "rotary embedding of the keys");
+  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && sdpa::prefill_supported(P, q, k_rot, v, out)) {
+    // the queries are rotated tile by tile in shared memory, from a cos / sin table
+    void* table = base_ws + L.table_off;
+    e = sdpa::launch_rope_table((long long)P.B * P.Lq, P.D, q_positions, base, table, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rotary table");
+    P.q_rope = static_cast<const float2*>(table);
+    const char* msg = nullptr;
+    e = sdpa::launch_prefill(P, q, k_rot, v, out, base_ws + L.q_off, s, &msg);
+    if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");
+    g_last_kernel = "prefill_tcgen05_rope";
+    return SDPA_OK;
+  }
+  void* q_rot = base_ws + L.q_off;
+  e = sdpa::launch_rope(P.dtype, q, q_rot, (long long)P.B * P.Lq, P.H, P.D, q_positions, base, s);
+  if (e != cudaSuccess) return cuda_fail(e, "rotary embedding of the queries");
+  if (!generic_ok(P))
+    return fail(SDPA_ERR_UNSUPPORTED, "head sizes dqk=%d dv=%d exceed the SIMT kernel's limits (1024, 256)",
+                P.D, P.Dv);
+  e = sdpa::launch_generic(P, q_rot, k_rot, v, out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "generic attention launch");
+  g_last_kernel = "generic_simt";
   return SDPA_OK;
 }
 
@@ -361,6 +454,17 @@ sdpa_status sdpa_decode_with_cache(const sdpa_params* p, const void* q, const vo
                                    const void* v_new, void* k_cache, void* v_cache,
                                    const int32_t* cache_index, void* out, void* ws,
                                    size_t ws_bytes, struct CUstream_st* stream) {
+  return sdpa::decode_with_cache(p, q, k_new, v_new, k_cache, v_cache, cache_index, out, ws, ws_bytes,
+                                 (cudaStream_t)stream, false);
+}
+
+}  // extern "C"
+
+namespace sdpa {
+
+sdpa_status decode_with_cache(const sdpa_params* p, const void* q, const void* k_new, const void* v_new,
+                              void* k_cache, void* v_cache, const int32_t* cache_index, void* out, void* ws,
+                              size_t ws_bytes, cudaStream_t s, bool clear_status) {
   sdpa::Problem P;
   sdpa_status st = resolve(p, &P);
   if (st != SDPA_OK) return st;
@@ -377,8 +481,11 @@ sdpa_status sdpa_decode_with_cache(const sdpa_params* p, const void* q, const vo
   if (P.B == 0 || P.Lq == 0) return SDPA_OK;
   if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_index || !out)
     return fail(SDPA_ERR_INVALID_ARG, "decode pointers must not be NULL");
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = sdpa::launch_cache_update(k_cache, nullptr, k_new, nullptr, dtype_size(P.dtype), P.D,
+  // every argument is valid: only now may the status word be cleared (a caller-owned
+  // workspace keeps the caller's word as it is)
+  cudaError_t e = clear_status ? cudaMemsetAsync(ws, 0, kStatusBytes, s) : cudaSuccess;
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  e = sdpa::launch_cache_update(k_cache, nullptr, k_new, nullptr, dtype_size(P.dtype), P.D,
                                             P.Hkv, P.Lq, P.Lk, P.B, cache_index, static_cast<int*>(ws), s);
   if (e == cudaSuccess)
     e = sdpa::launch_cache_update(nullptr, v_cache, nullptr, v_new, dtype_size(P.dtype), P.Dv, P.Hkv,
@@ -399,6 +506,10 @@ sdpa_status sdpa_decode_with_cache(const sdpa_params* p, const void* q, const vo
   g_last_kernel = "generic_simt";
   return SDPA_OK;
 }
+
+}  // namespace sdpa
+
+extern "C" {
 
 size_t build_block_mask_info_size(int32_t nheads, int32_t q_len, int32_t kv_len, int32_t bq,
                                   int32_t bk) {
@@ -470,5 +581,13 @@ sdpa_status sdpa_read_device_status(void* ws, struct CUstream_st* stream) {
 const char* sdpa_last_error(void) { return g_last_error.c_str(); }
 
 const char* sdpa_last_kernel(void) { return g_last_kernel; }
+
+int sdpa_debug_checks(void) {
+#ifdef SDPA_DEBUG_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 }  // extern "C"

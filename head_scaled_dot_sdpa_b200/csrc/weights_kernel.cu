@@ -8,9 +8,11 @@
 // [batch][nheads][q_len][kv_len], in the input type. A row with no attended key has NaN weights
 // and output; a row past q_lengths has zero weights and output.
 //
-// The dropout draw is counter-based: u = top 53 bits of fmix64(seed + fmix64(index)) / 2^53,
-// where fmix64 is the 64-bit finalizer of Austin Appleby's MurmurHash3 and index is the
-// weight's row-major position. A weight is kept when u >= p, compared in double precision.
+// The dropout draw is counter-based: the weights' row-major positions are taken four at a
+// time, the group index / 4 gets r = fmix64(seed + fmix64(index / 4)) (fmix64: the 64-bit
+// finalizer of Austin Appleby's MurmurHash3), and the weight at `index` takes the 16-bit field
+// number index % 4 of r (lowest first) as u in [0, 2^16); it is kept when
+// u >= ceil(p * 2^16), an integer comparison.
 //
 // Two kernels:
 //  - weights_mma_kernel (bf16/fp16, head_dim = v_head_dim = 64 or 128): one CTA per
@@ -28,19 +30,10 @@ using namespace tiles;
 constexpr int kRows = 64;  // query rows per CTA
 constexpr int kKeys = 64;  // keys per tile
 
-__device__ __forceinline__ unsigned long long fmix64(unsigned long long k) {
-  k ^= k >> 33;
-  k *= 0xff51afd7ed558ccdULL;
-  k ^= k >> 33;
-  k *= 0xc4ceb9fe1a85ec53ULL;
-  k ^= k >> 33;
-  return k;
-}
-
-// Whether the dropout keeps the weight at row-major position `index`.
-__device__ __forceinline__ bool keep(unsigned long long seed, unsigned long long index, double p) {
-  const double u = (double)(fmix64(seed + fmix64(index)) >> 11) * (1.0 / 9007199254740992.0);
-  return u >= p;
+// Whether the dropout keeps the weight at row-major position `index` (threshold =
+// ceil(p * 2^16)).
+__device__ __forceinline__ bool keep(unsigned long long seed, unsigned long long index, unsigned threshold) {
+  return (dropout_keep4(dropout_group_draw(seed, index >> 2), threshold) >> (index & 3)) & 1u;
 }
 
 // The logit of (i, j) in log2 units: (scale q.k + bias) * log2(e), from the raw dot product.
@@ -78,6 +71,7 @@ weights_mma_kernel(Problem P, const T* __restrict__ q, const T* __restrict__ k, 
   const int rl = warp * 16 + gq, rh = rl + 8;
   const int il = i0 + rl, ih = i0 + rh;
   const float inv_keep = (float)(1.0 / (1.0 - drop_p));
+  const unsigned drop_thr = (unsigned)ceil(drop_p * 65536.0);
   float acc[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -194,7 +188,7 @@ weights_mma_kernel(Problem P, const T* __restrict__ q, const T* __restrict__ k, 
             w = exp2f(logit2(P, b, h, i, j, s[n][e]) - L);
             if (drop_p > 0.0) {
               const unsigned long long idx = (((unsigned long long)b * P.H + h) * P.Lq + i) * P.Lk + j;
-              w = keep(seed, idx, drop_p) ? w * inv_keep : 0.f;
+              w = keep(seed, idx, drop_thr) ? w * inv_keep : 0.f;
             }
           }
           s[n][e] = w;
@@ -298,6 +292,7 @@ weights_simt_kernel(Problem P, const T* __restrict__ q, const T* __restrict__ k,
     return;
   }
   const float L = m + log2f(l), inv_keep = (float)(1.0 / (1.0 - drop_p));
+  const unsigned drop_thr = (unsigned)ceil(drop_p * 65536.0);
   float o[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) o[u] = 0.f;
@@ -310,7 +305,7 @@ weights_simt_kernel(Problem P, const T* __restrict__ q, const T* __restrict__ k,
         w = exp2f(x - L);
         if (drop_p > 0.0) {
           const unsigned long long idx = (((unsigned long long)b * P.H + h) * P.Lq + i) * P.Lk + j;
-          w = keep(seed, idx, drop_p) ? w * inv_keep : 0.f;
+          w = keep(seed, idx, drop_thr) ? w * inv_keep : 0.f;
         }
       }
       wrow[j] = from_f32<T>(w);

@@ -207,14 +207,24 @@ SDPA_API sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed
  *  - weights (device, caller-owned, p->dtype) gets the page's (kv_len, q_len, nheads, batch)
  *    order, row-major [batch][nheads][q_len][kv_len], after the dropout. A row with no attended
  *    key has NaN weights and output. A row past q_lengths has zero weights and output.
- *  - The dropout keeps w_ij, divided by 1 - drop_p, when u >= drop_p, and otherwise sets it
- *    to 0. Here u = (fmix64(seed + fmix64(index)) >> 11) / 2^53, compared in double, where
- *    fmix64 is the 64-bit finalizer of MurmurHash3 and index is the weight's row-major
- *    position. drop_p must be in [0, 1), and 0 means no dropout.
+ *  - The dropout keeps w_ij, divided by 1 - drop_p, when its draw u >= ceil(drop_p * 2^16),
+ *    and otherwise sets it to 0. The weights' row-major positions are taken four at a time:
+ *    the group index / 4 gets r = fmix64(seed + fmix64(index / 4)), fmix64 being the 64-bit
+ *    finalizer of MurmurHash3, and u is the 16-bit field index % 4 of r (lowest first). So a
+ *    weight is kept with probability 1 - ceil(drop_p * 2^16) / 2^16, within 2^-16 of
+ *    1 - drop_p. drop_p must be in [0, 1), and 0 means no dropout.
  *  - out = weights · v.
- *  - The workspace holds only the status word (at least 256 bytes).
- *  - Kernels. mma.sync tiles for bf16/fp16 with dqk = dv = 64 or 128. A SIMT kernel handles
- *    the rest, or runs when SDPA_FLAG_GENERIC_KERNEL is set. */
+ *  - The workspace holds the status word and one float per query row (the row's log-sum-exp):
+ *    sdpa_weights_workspace_size(p) bytes.
+ *  - Kernels. bf16/fp16 with dqk = dv = 64 or 128, no bias, mask or block_info, kv_len a
+ *    multiple of 8 and 16-byte aligned arrays run on the tcgen05 prefill kernel: the forward
+ *    (writing the row log-sum-exp), a kernel that writes the weights of the key tiles beyond
+ *    each query tile's causal / kv_lengths bound (0, or NaN for a row with no key), then the
+ *    weights pass, which recomputes the logits on the tensor cores, stores the weights of the
+ *    visited tiles with 16-byte stores and accumulates out from the dropped weights. Other
+ *    bf16/fp16 calls with dqk = dv = 64 or 128 take mma.sync tiles; a SIMT kernel handles the
+ *    rest, or runs when SDPA_FLAG_GENERIC_KERNEL is set. */
+SDPA_API size_t sdpa_weights_workspace_size(const sdpa_params* p);
 SDPA_API sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop_p, uint64_t seed, const void* q,
                                                const void* k, const void* v, void* out, void* weights, void* ws,
                                                size_t ws_bytes, struct CUstream_st* stream);
@@ -228,11 +238,34 @@ SDPA_API sdpa_status sdpa_forward_with_weights(const sdpa_params* p, double drop
  *    rows = batch * seq_len). out may be x (in place).
  *  - positions: device int32[rows], the position of each row. With a KV cache this is the
  *    absolute position, cache index + t.
- *  - d must be even and base > 0 (10000 is the usual value). The angle and the rotation are
- *    taken in double precision.
+ *  - d must be even, at most 8192 (SDPA_ERR_UNSUPPORTED beyond), and base > 0 (10000 is the
+ *    usual value). The frequencies and the angle, reduced to [-pi, pi], are taken in double
+ *    precision; CUDA's sincosf evaluates the reduced angle and the rotation is in fp32.
  *  - One elementwise kernel; no workspace. */
 SDPA_API sdpa_status sdpa_rope(const void* x, void* out, sdpa_dtype dtype, int64_t rows, int32_t nheads, int32_t d,
                                const int32_t* positions, double base, struct CUstream_st* stream);
+
+/* Attention with the rotary position embedding of the queries and keys (the form of sdpa_rope)
+ * folded into the call: out = sdpa_forward(p, rope(q, q_positions), rope(k, k_positions), v).
+ * The Keras thread "MultiHeadAttention is missing a position_bias call argument" applies the
+ * rotary embedding to the query and key right before the attention; here q and k are read
+ * as given and not modified.
+ *  - q_positions: device int32[batch * q_len], k_positions: device int32[batch * kv_len], the
+ *    position of each row (the absolute position; with a cache, cache index + t). base > 0.
+ *  - Every argument of sdpa_forward applies to the rotated arrays; qk_head_dim must be even.
+ *  - The workspace (sdpa_rope_workspace_size(p) bytes) holds the status word, the rotated keys
+ *    (one pass over k: every query tile of a key/value head reads them), a cos / sin table of
+ *    the query rows and room for rotated queries.
+ *  - Kernels. Where sdpa_forward takes the tcgen05 kernel, a table kernel computes the query
+ *    angles' cos / sin and the attention kernel rotates each Q tile in shared memory after
+ *    its TMA load, before the first QK^T MMA reads it, so the rotated queries never go to
+ *    memory. Otherwise the queries are rotated into the workspace and the SIMT kernel runs.
+ *    The rotated values are rounded to the input type, as sdpa_rope's output is. */
+SDPA_API size_t sdpa_rope_workspace_size(const sdpa_params* p);
+SDPA_API sdpa_status sdpa_forward_rope(const sdpa_params* p, const int32_t* q_positions,
+                                       const int32_t* k_positions, double base, const void* q,
+                                       const void* k, const void* v, void* out, void* ws,
+                                       size_t ws_bytes, struct CUstream_st* stream);
 
 /* Workspace bytes sdpa_backward needs for these params (256-byte aligned; 0 if invalid). */
 SDPA_API size_t sdpa_backward_workspace_size(const sdpa_params* p);
@@ -266,8 +299,9 @@ SDPA_API sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const vo
  * kv_lengths[b] = cache_index[b] + n_new. Here p->q_len = n_new, p->kv_len = capacity,
  * p->causal must be SDPA_CAUSAL_BOTTOM_RIGHT and q_lengths, kv_lengths, bias, mask and
  * block_info must be NULL. cache_index is a device int32[batch]; a value outside
- * [0, capacity - n_new] skips that sequence's write and attention (its output rows are left
- * as they were) and sets SDPA_ERR_DEVICE_CHECK in the status word. */
+ * [0, capacity - n_new] skips that sequence's cache write and attention, writes NaN to its
+ * output rows (so the failure shows in the result) and sets SDPA_ERR_DEVICE_CHECK in the
+ * status word. */
 SDPA_API sdpa_status sdpa_decode_with_cache(const sdpa_params* p, const void* q, const void* k_new,
                                    const void* v_new, void* k_cache, void* v_cache,
                                    const int32_t* cache_index, void* out, void* ws,
@@ -286,15 +320,28 @@ SDPA_API sdpa_status sdpa_decode_with_cache(const sdpa_params* p, const void* q,
  *    current. Make that first call before any stream capture.
  *  - Every call on a device shares the one array. Calls that overlap on the GPU (other streams,
  *    other host threads) race on it: serialise them.
- *  - The device status word sits in the array and is cleared at the start of each call. The
- *    caller cannot read it. An out-of-range cache_index still skips that sequence.
+ *  - Invalid arguments return a status before anything is queued, as for
+ *    sdpa_decode_with_cache. A valid call first clears the device status word, which sits in
+ *    the array, and then runs the same kernels. An out-of-range cache_index skips that
+ *    sequence, writes NaN to its output rows and sets SDPA_ERR_DEVICE_CHECK in that word;
+ *    sdpa_read_static_status() returns and clears it.
+ *  - 40 MiB holds the partials of a bf16/fp16 decode step of 64 sequences x 8 key/value
+ *    heads x capacity 8192 at head_dim 128 (34.1 MB). A call whose sdpa_workspace_size(p)
+ *    exceeds it is rejected (first point above).
  *  - Nothing is allocated. No cudaMalloc, cudaFree or allocating library routine is called. */
-#define SDPA_STATIC_SCRATCH_BYTES (32u << 20)
+#define SDPA_STATIC_SCRATCH_BYTES (40u << 20)
 SDPA_API sdpa_status sdpa_decode_with_cache_static(const sdpa_params* p, const void* q,
                                                    const void* k_new, const void* v_new,
                                                    void* k_cache, void* v_cache,
                                                    const int32_t* cache_index, void* out,
                                                    struct CUstream_st* stream);
+
+/* The device status word of sdpa_decode_with_cache_static on the current device: synchronises
+ * `stream`, returns SDPA_OK or the first device error recorded since the last call that
+ * cleared it (every static call clears it when it starts, so this reports the most recent
+ * static call), and resets it to SDPA_OK. SDPA_OK if no static call has run on this device.
+ * Like the static call it allocates nothing (no counterpart in the paper). */
+SDPA_API sdpa_status sdpa_read_static_status(struct CUstream_st* stream);
 
 /* Writes k_new/v_new [batch][n_new][nkvheads][d] of `dtype` into the caches
  * [batch][capacity][nkvheads][d] at rows index[b] + t, t < n_new (index: device
@@ -337,6 +384,15 @@ SDPA_API const char* sdpa_last_error(void);
  * ("generic_simt", "prefill_tcgen05", "decode_splitkv", "weights_mma", "weights_simt",
  * "backward_mma", "backward_simt"). */
 SDPA_API const char* sdpa_last_kernel(void);
+
+/* 1 in the range-checked build of the library (compiled with SDPA_DEBUG_CHECKS, shipped as
+ * libsdpa_debug.so), 0 in the normal one. In the range-checked build every device-side index the
+ * kernels take from data (block-row counts and lists, partial-bit addresses, TMA tile
+ * coordinates, cache and split indices, output rows) is checked before use; a violation sets
+ * SDPA_ERR_DEVICE_CHECK in the status word and the access is skipped (or, for a TMA
+ * coordinate, clamped into the array), so a bad input is reported instead of faulting. It is
+ * the stand-in for a memory checker and costs speed. */
+SDPA_API int sdpa_debug_checks(void);
 
 #ifdef __cplusplus
 }

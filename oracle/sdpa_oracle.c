@@ -212,9 +212,12 @@ int oracle_rope(const double* x, int64_t rows, int64_t nheads, int64_t d, const 
   return ORACLE_OK;
 }
 
-/* Counter-based uniform draw for dropout: the 64-bit finalizer of Austin Appleby's MurmurHash3
- * ("fmix64"), applied twice, to the element's linear index (b, h, i, j) and then to that plus
- * the seed. The top 53 bits give u in [0, 1). */
+/* Counter-based dropout draw. The weights' linear indices (b, h, i, j), row-major, are taken
+ * four at a time: the group index / 4 gets one 64-bit value from the 64-bit finalizer of Austin
+ * Appleby's MurmurHash3 ("fmix64"), applied to the group and then to that plus the seed, and
+ * the weight at `index` takes its 16-bit field number index % 4 (lowest first) as an integer u
+ * in [0, 2^16). The weight is kept when u >= threshold = ceil(drop_p * 2^16): with probability
+ * 1 - threshold / 2^16, within 2^-16 of 1 - drop_p. */
 static uint64_t fmix64(uint64_t k) {
   k ^= k >> 33;
   k *= 0xff51afd7ed558ccdULL;
@@ -223,8 +226,10 @@ static uint64_t fmix64(uint64_t k) {
   k ^= k >> 33;
   return k;
 }
-static double dropout_uniform(uint64_t seed, uint64_t index) {
-  return (double)(fmix64(seed + fmix64(index)) >> 11) * (1.0 / 9007199254740992.0);
+static int dropout_keep(uint64_t seed, uint64_t index, uint32_t threshold) {
+  const uint64_t r = fmix64(seed + fmix64(index >> 2));
+  const uint32_t u = (uint32_t)(r >> (16 * (index & 3))) & 0xFFFFu;
+  return u >= threshold;
 }
 
 /* scaled_dot_product_attention_with_weights (the entry's "See also": the attention weights too)
@@ -232,7 +237,7 @@ static double dropout_uniform(uint64_t seed, uint64_t index) {
  * right after the softmax). The weights are materialized (paragraph "Fused implementation":
  * any call with an fdrop takes the materialized implementation):
  *   w_ij = softmax_j(scale q_i.k_j + bias_ij, masked)
- *   w'_ij = w_ij / (1 - drop_p) where u(seed, b, h, i, j) >= drop_p, else 0
+ *   w'_ij = w_ij / (1 - drop_p) where the draw of (b, h, i, j) keeps it, else 0
  *   out_i = sum_j w'_ij v_j
  * and `weights` receives w' in the page's (kv_len, q_len, nheads, batch) order, which is
  * row-major [batch][nheads][q_len][kv_len]. A row with no attended key has NaN weights and a
@@ -296,10 +301,11 @@ int oracle_sdpa_forward_with_weights(const oracle_sdpa_problem* p, const double*
       z += wrow[j];
     }
     const uint64_t base = (uint64_t)(((b * H + h) * Lq + i) * Lk);
+    const uint32_t thr = (uint32_t)ceil(drop_p * 65536.0);
     for (int64_t j = 0; j < Lk; ++j) {
       double w = wrow[j] / z;
       if (drop_p > 0.0)
-        w = (dropout_uniform(seed, base + (uint64_t)j) >= drop_p) ? w / (1.0 - drop_p) : 0.0;
+        w = dropout_keep(seed, base + (uint64_t)j, thr) ? w / (1.0 - drop_p) : 0.0;
       wrow[j] = w;
       if (w == 0.0) continue;
       const double* vj = v + ((b * Lk + j) * Hkv + g) * Dv;

@@ -492,6 +492,10 @@ def dropout_keeps_one_minus_p_unbiased(lib):
     assert abs(kept.mean() - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
     _close(w[kept], w0[kept] / (1 - p), 1e-15)
     _close(out, np.einsum("bhij,bjhe->bihe", w, np.repeat(v, 2, axis=2)))
+    # neighbouring weights draw independently, also the four that share one 64-bit hash
+    a, c = kept[..., :-1].ravel(), kept[..., 1:].ravel()
+    both = (a & c).mean()
+    assert abs(both - (1 - p) ** 2) < 5 * math.sqrt((1 - p) ** 2 * (1 - (1 - p) ** 2) / a.size)
     _, w2 = oracle.sdpa_forward_with_weights(q, k, v, drop_p=p, seed=8, lib=lib)
     assert ((w2 != 0) != kept).mean() > 0.3
     acc = np.zeros((1, 10, 4, 50))

@@ -28,6 +28,27 @@ def test_every_declared_function_is_exported():
     assert set(names) <= exported
 
 
+def test_range_checked_build_differs_and_reports_itself():
+    """libsdpa_debug.so is the same sources compiled with SDPA_DEBUG_CHECKS: it exports the same
+    entry points, says so through sdpa_debug_checks(), and its kernels are different code."""
+    debug = os.path.join(os.path.dirname(sdpa.LIB_PATH), "libsdpa_debug.so")
+    normal = os.path.join(os.path.dirname(sdpa.LIB_PATH), "libsdpa.so")
+    assert os.path.exists(debug), "build it with head_scaled_dot_sdpa_b200/build.py --debug-checks"
+    libs = {path: ctypes.CDLL(path) for path in (normal, debug)}
+    for lib in libs.values():
+        lib.sdpa_debug_checks.restype = ctypes.c_int
+        for n in declared_functions():
+            assert hasattr(lib, n), n
+    assert libs[normal].sdpa_debug_checks() == 0
+    assert libs[debug].sdpa_debug_checks() == 1
+    objs = os.path.join(ROOT, "_build")
+    a = os.path.join(objs, "sdpa", "prefill_bf16_d128.cu.o")
+    b = os.path.join(objs, "sdpa_debug", "prefill_bf16_d128.cu.o")
+    if os.path.exists(a) and os.path.exists(b):
+        assert open(a, "rb").read() != open(b, "rb").read()
+    assert open(normal, "rb").read() != open(debug, "rb").read()
+
+
 def test_struct_layout_matches_binding(tmp_path):
     src = tmp_path / "layout.c"
     fields = [f[0] for f in sdpa.Params._fields_]

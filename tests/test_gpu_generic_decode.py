@@ -118,6 +118,30 @@ def test_decode_with_cache(dtype, D, H, Hkv, n_new, generic):
     assert sdpa.read_device_status() == sdpa.SDPA_OK
 
 
+@pytest.mark.parametrize("generic", [False, True])
+def test_decode_bad_index_nan_rows(generic):
+    """A cache index out of range skips that sequence (cache untouched), writes NaN to its output
+    rows and sets the status word; the other sequences match the oracle."""
+    B, cap, H, Hkv, D = 4, 300, 8, 2, 128
+    q, kn, vn, kc, vc, idx = _decode_case(B, cap, H, Hkv, D, 2, torch.bfloat16, seed=11)
+    idx = idx.copy()
+    idx[1] = cap - 1  # a 2-token write would end past the capacity
+    idx[3] = -1
+    kc_d, vc_d = kc.to(DEV), vc.to(DEV)
+    ws = sdpa.Workspace(DEV)
+    out = sdpa.sdpa_decode_with_cache(q.to(DEV), kn.to(DEV), vn.to(DEV), kc_d, vc_d, torch.from_numpy(idx),
+                                      generic=generic, workspace=ws)
+    assert sdpa.read_device_status(ws) == sdpa.SDPA_ERR_DEVICE_CHECK
+    got = out.cpu()
+    for b in (1, 3):
+        assert torch.isnan(got[b].float()).all()
+        np.testing.assert_array_equal(f64(kc_d[b]), f64(kc[b]))
+    good = np.array([0, 2])
+    want, _, _ = oracle.sdpa_decode_with_cache(f64(q[good]), f64(kn[good]), f64(vn[good]), f64(kc[good]),
+                                               f64(vc[good]), idx[good])
+    assert_matches(got[good], want, 1e-2, "decode next to bad indices")
+
+
 def test_decode_split_boundaries():
     """Lengths at and around the split size, and a single key."""
     B, cap, H, Hkv, D = 8, 2048, 8, 2, 128

@@ -38,7 +38,9 @@ MUTANTS = {
     "rope_sin_sign": ("o[c] = x0 * cos(a) - x1 * sin(a);", "o[c] = x0 * cos(a) + x1 * sin(a);"),
     "rope_frequency_exponent": ("pow(base, -2.0 * (double)c / (double)d)", "pow(base, -1.0 * (double)c / (double)d)"),
     "weights_dropout_unscaled": ("? w / (1.0 - drop_p) : 0.0", "? w : 0.0"),
-    "weights_dropout_inverted": ("base + (uint64_t)j) >= drop_p)", "base + (uint64_t)j) < drop_p)"),
+    "weights_dropout_inverted": ("dropout_keep(seed, base + (uint64_t)j, thr) ?", "!dropout_keep(seed, base + (uint64_t)j, thr) ?"),
+    "weights_dropout_same_draw_per_group": ("fmix64(index >> 2));\n  const uint32_t u = (uint32_t)(r >> (16 * (index & 3)))",
+                                            "fmix64(index >> 2));\n  const uint32_t u = (uint32_t)(r >> 0)"),
     "weights_head_batch_swapped": ("double* wrow = weights + ((b * H + h) * Lq + i) * Lk;",
                                    "double* wrow = weights + ((h * B + b) * Lq + i) * Lk;"),
     "backward_delta_sign": ("x[j] * (dw[j] - wdw)", "x[j] * (dw[j] + wdw)"),
