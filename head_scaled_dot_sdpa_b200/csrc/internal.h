@@ -51,9 +51,9 @@ struct Problem {
   unsigned long long drop_seed;
   unsigned drop_thr;
   float inv_keep;
-  // rotary embedding of the Q tiles in shared memory (sdpa_forward_rope): cos / sin of each
-  // query row's angles, float2 [B * Lq][D / 2]; null when the queries are not rotated
-  const float2* q_rope;
+  // rotary embedding of the Q tiles in shared memory (sdpa_forward_rope): (cos, sin) of each
+  // query row's angles as fp16 pairs, [B * Lq][D / 2] 32-bit words; null when not rotated
+  const uint32_t* q_rope;
   int* status;               // device status word (never null when a kernel runs)
   unsigned long long wait_timeout_ns;  // bound on every mbarrier wait of the tcgen05 kernel
   int selftest_stall;                  // SDPA_FLAG_SELFTEST_STALL
@@ -121,7 +121,7 @@ cudaError_t launch_weights(const Problem& P, bool tiles, const void* q, const vo
 // Rotary position embedding of [rows][nheads][d] rows (out may alias x).
 cudaError_t launch_rope(int dtype, const void* x, void* out, long long rows, int nheads, int d,
                         const int32_t* positions, double base, cudaStream_t stream);
-// cos / sin of the rotary angles of `rows` positions: float2 table[rows][d / 2].
+// (cos, sin) of the rotary angles of `rows` positions as fp16 pairs: table[rows][d / 2].
 cudaError_t launch_rope_table(long long rows, int d, const int32_t* positions, double base, void* table,
                               cudaStream_t stream);
 bool prefill_supported(const Problem& P, const void* q, const void* k, const void* v,

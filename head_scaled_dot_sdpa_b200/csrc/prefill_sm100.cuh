@@ -63,9 +63,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 bytes (64 16-bit columns)
 constexpr int kNone = 1 << 30;
 constexpr int kUnitSlots = 4;        // ring of unit indices handed from the producer to the others
-constexpr int kUnitConsumers = 10;   // the two MMA warps and the 8 softmax warps (+ the rope warp)
+constexpr int kUnitConsumers = 10;   // the two MMA warps and the 8 softmax warps
 constexpr int kMmaWarpA = 9, kMmaWarpB = 11;  // MMA issuers of tile A and tile B
-constexpr int kRopeWarp = 10;        // rotates the Q tiles in shared memory when P.q_rope is set
 constexpr int kSchedWord = 16;       // int offset in the status area of the unit counter (+1: done)
 
 // bias / mask variants compiled into the kernel
@@ -78,20 +77,20 @@ enum { kMaskNone = 0, kMaskDense = 1, kMaskBits = 2 };
 // weights 2^(x - lse) of the visited key tiles, dropped out and stored, and out = sum w' v.
 enum { kModeForward = 0, kModeWeights = 2 };
 
-// Shared-memory plan. With bias tiles (kBT, head_dim 64) each query tile has kBiasSlots bias
-// tiles in flight, so the next key tile's bias streams in from HBM while the current one is
-// read; the K and V rings then keep 2 stages each to make room.
+// Shared-memory plan: the Q tiles of the two query tiles, the K and V rings, and with bias
+// tiles (kBT, head_dim 64) one bias tile per query tile. (A third Q slot, so that the next
+// unit's first Q tile loads a whole unit ahead, and two bias tiles in flight per query tile
+// were measured on B200 and were 1-2 % slower; the slot counts stay parameters.)
 template <int D, bool kBT = false>
 struct Cfg {
   static constexpr int kRegions = D / 64;
   static constexpr int kTileBytes = kRegions * kRegionBytes;
-  static constexpr int kKStages = (D == 128 || kBT) ? 2 : 4;
-  static constexpr int kVStages = (D == 128 || kBT) ? 2 : 4;
+  static constexpr int kKStages = D == 128 ? 2 : 4;
+  static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr int kBiasTileBytes = 128 * 128 * 2;
-  static constexpr int kBiasSlots = 2;  // per query tile
+  static constexpr int kBiasSlots = 1;  // per query tile
   // Q tiles: a ring shared by the two query tiles of the units, in the order A, B, A, B, ...
-  // With a third slot the next unit's tile A loads while the current unit still holds both.
-  static constexpr int kQSlots = kBT ? 2 : 3;
+  static constexpr int kQSlots = 2;
   static constexpr int kBiasBytes = kBT ? 2 * kBiasSlots * kBiasTileBytes : 0;
   static constexpr int kBarriers =
       3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots;
@@ -247,6 +246,46 @@ __device__ __noinline__ void rescale_o(uint32_t taddr, float a) {
   tmem_wait_st();
 }
 
+// Rotary embedding of row r of a Q tile in shared memory (128-byte swizzle: logical 16-byte
+// chunk x of row r is stored at chunk x ^ (r % 8)): the pair (c, c + D/2) rotated by the angle
+// whose (cos, sin) fp16 pair is table[c]. Out of line, like rescale_o, so that the softmax
+// loop's code and registers stay as they are when no rotation is asked for.
+template <typename T, int D>
+__device__ __noinline__ void rotate_q_row(uint8_t* tile, int r, const uint32_t* table) {
+  constexpr int kHalf = D / 2, kPairChunks = kHalf / 8;
+  const uint4* trow = reinterpret_cast<const uint4*>(table);
+  uint4 tab[2 * kPairChunks];
+#pragma unroll
+  for (int z = 0; z < 2 * kPairChunks; ++z) tab[z] = trow[z];
+#pragma unroll
+  for (int x = 0; x < kPairChunks; ++x) {
+    uint8_t* lo = tile + r * 128 + ((x ^ (r & 7)) << 4);
+    uint8_t* hi = D == 128 ? lo + kRegionBytes : tile + r * 128 + (((x + 4) ^ (r & 7)) << 4);
+    uint4 a = *reinterpret_cast<uint4*>(lo), b = *reinterpret_cast<uint4*>(hi);
+    uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
+    uint32_t* pb = reinterpret_cast<uint32_t*>(&b);
+    const uint32_t* cs = reinterpret_cast<const uint32_t*>(&tab[2 * x]);  // 8 (cos, sin) pairs
+#pragma unroll
+    for (int z = 0; z < 4; ++z) {
+      float y0[2], y1[2];
+#pragma unroll
+      for (int y = 0; y < 2; ++y) {
+        const uint16_t la = (uint16_t)(pa[z] >> (16 * y)), lb = (uint16_t)(pb[z] >> (16 * y));
+        const float x0 = to_f32(*reinterpret_cast<const T*>(&la));
+        const float x1 = to_f32(*reinterpret_cast<const T*>(&lb));
+        const __half2 t2 = *reinterpret_cast<const __half2*>(&cs[2 * z + y]);
+        const float cv = __low2float(t2), sv = __high2float(t2);
+        y0[y] = x0 * cv - x1 * sv;
+        y1[y] = x1 * cv + x0 * sv;
+      }
+      pa[z] = std::is_same<T, __half>::value ? pack_f16x2(y0[0], y0[1]) : pack_bf16x2(y0[0], y0[1]);
+      pb[z] = std::is_same<T, __half>::value ? pack_f16x2(y1[0], y1[1]) : pack_bf16x2(y1[0], y1[1]);
+    }
+    *reinterpret_cast<uint4*>(lo) = a;
+    *reinterpret_cast<uint4*>(hi) = b;
+  }
+}
+
 template <typename T, int D, int kBias, int kMask, int kMode = kModeForward>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __restrict__ out, int n_units) {
@@ -288,7 +327,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     for (int x = 0; x < C::kQSlots; ++x) {
       mbar_init(&q_full[x], 1);
       mbar_init(&q_empty[x], 1);
-      mbar_init(&q_rot[x], 1);
+      mbar_init(&q_rot[x], 4);  // one arrive per softmax warp of the tile
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
@@ -306,7 +345,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     mbar_init(drain, 2);
     for (int k = 0; k < kUnitSlots; ++k) {
       mbar_init(&unit_full[k], 1);
-      mbar_init(&unit_empty[k], kUnitConsumers + (P.q_rope ? 1 : 0));
+      mbar_init(&unit_empty[k], kUnitConsumers);
     }
     *abort_flag = 0;
     issued[0] = 0;
@@ -649,74 +688,6 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         base_o += groups_o;
       }
     }();
-  } else if (warp == kRopeWarp) {
-    // ------------------------------------------------------------------ rotary embedding of Q
-    // Each Q tile, once loaded, is rotated in shared memory: the pair (c, c + D/2) of query row
-    // i by the angle whose cos / sin P.q_rope holds for row b * Lq + i. A lane takes 16-byte
-    // chunks (8 pairs) of one row; 128-byte swizzle: logical chunk x of row r is stored at
-    // chunk x ^ (r % 8). The writes are made visible to the tensor core (async proxy) before
-    // the tile is released to its MMA warp.
-    if (P.q_rope) [&] {
-      constexpr int kHalf = D / 2;
-      constexpr int kPairChunks = kHalf / 8;  // 16-byte chunk pairs per row
-      uint32_t qi = 0;
-      for (uint32_t kq = 0;; ++kq) {
-        int u;
-        if (!next_unit(kq, u)) return;
-        if (u >= n_units) break;
-        const Unit w = make_unit(P, u);
-        if (w.t[0].n == 0 && w.t[1].n == 0) continue;
-#pragma unroll 1
-        for (int s = 0; s < 2; ++s) {
-          const QTile qt = s ? w.t[1] : w.t[0];
-          if (qt.n == 0) continue;
-          const int qs = (int)(qi % C::kQSlots);
-          if (!wait_all(&q_full[qs], (qi / C::kQSlots) & 1)) return;
-          uint8_t* tile = q_smem + qs * C::kTileBytes;
-          const int rows = min(kBlockM, P.Lq - qt.i0);  // rows past the array are zeros
-#pragma unroll 1
-          for (int item = lane; item < rows * kPairChunks; item += 32) {
-            const int r = item / kPairChunks, x = item % kPairChunks;
-            // chunk x of the first half pairs with chunk x of the second half (D = 128: the
-            // second 64-column region; D = 64: chunk x + 4 of the one region)
-            uint8_t* lo = tile + r * 128 + ((x ^ (r & 7)) << 4);
-            uint8_t* hi = D == 128 ? lo + kRegionBytes : tile + r * 128 + (((x + 4) ^ (r & 7)) << 4);
-            const float4* cs = reinterpret_cast<const float4*>(
-                P.q_rope + ((long long)w.b * P.Lq + qt.i0 + r) * kHalf + 8 * x);
-            float tc[16];
-#pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              const float4 f = cs[z];
-              tc[4 * z] = f.x; tc[4 * z + 1] = f.y; tc[4 * z + 2] = f.z; tc[4 * z + 3] = f.w;
-            }
-            uint4 a = *reinterpret_cast<uint4*>(lo), b = *reinterpret_cast<uint4*>(hi);
-            uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
-            uint32_t* pb = reinterpret_cast<uint32_t*>(&b);
-#pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              float x0[2], x1[2];
-#pragma unroll
-              for (int y = 0; y < 2; ++y) {
-                const uint16_t la = (uint16_t)(pa[z] >> (16 * y)), lb = (uint16_t)(pb[z] >> (16 * y));
-                x0[y] = to_f32(*reinterpret_cast<const T*>(&la));
-                x1[y] = to_f32(*reinterpret_cast<const T*>(&lb));
-              }
-              const float c0 = tc[4 * z], s0 = tc[4 * z + 1], c1 = tc[4 * z + 2], s1 = tc[4 * z + 3];
-              const float y00 = x0[0] * c0 - x1[0] * s0, y10 = x1[0] * c0 + x0[0] * s0;
-              const float y01 = x0[1] * c1 - x1[1] * s1, y11 = x1[1] * c1 + x0[1] * s1;
-              pa[z] = std::is_same<T, __half>::value ? pack_f16x2(y00, y01) : pack_bf16x2(y00, y01);
-              pb[z] = std::is_same<T, __half>::value ? pack_f16x2(y10, y11) : pack_bf16x2(y10, y11);
-            }
-            *reinterpret_cast<uint4*>(lo) = a;
-            *reinterpret_cast<uint4*>(hi) = b;
-          }
-          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-          __syncwarp();
-          if (elected) mbar_arrive(&q_rot[qs]);
-          ++qi;
-        }
-      }
-    }();
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax + epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
@@ -727,12 +698,30 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
       uint32_t sc = 0, oc = 0, bcs = 0;  // S tiles, units, bias tiles seen
+      uint32_t qi = 0;                   // Q tiles of both streams so far (ring position)
       for (uint32_t kq = 0;; ++kq) {
         int u;
         if (!next_unit(kq, u)) return;
         if (u >= n_units) break;
         const Unit w = make_unit(P, u);
         const QTile qt = s ? w.t[1] : w.t[0];
+        const uint32_t my_qi = qi + ((s == 1 && w.t[0].n > 0) ? 1u : 0u);
+        qi += (w.t[0].n > 0 ? 1u : 0u) + (w.t[1].n > 0 ? 1u : 0u);
+        if (P.q_rope && qt.n > 0) {
+          // Rotary embedding of this thread's query row in the tile's Q slot, once the tile
+          // has landed: the pair (c, c + D/2) by the angle whose (cos, sin) the table holds
+          // as fp16 for row b * Lq + i. 128-byte swizzle: logical 16-byte chunk x of row r
+          // is stored at chunk x ^ (r % 8). The writes are made visible to the tensor core
+          // (async proxy) before the warp releases the tile to its MMA warp.
+          const int qslot = (int)(my_qi % C::kQSlots);
+          if (!wait_all(&q_full[qslot], (my_qi / C::kQSlots) & 1)) return;
+          if (qt.i0 + r < P.Lq)
+            rotate_q_row<T, D>(q_smem + qslot * C::kTileBytes, r,
+                               P.q_rope + ((long long)w.b * P.Lq + qt.i0 + r) * (D / 2));
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&q_rot[qslot]);
+        }
         if (qt.i0 == kNone) continue;  // the unit has no tile B
         const int i = qt.i0 + r;
         T* orow = out + ((w.o0 + i) * P.H + qt.h) * D;
@@ -881,6 +870,50 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
 #pragma unroll
               for (int e = 0; e < 32; e += 2)
                 mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
+          } else if constexpr (kBias != kBiasNone && kMask != kMaskDense) {
+            // With a bias: the logits stay in natural units, x = s * scale + b (one packed FMA
+            // per pair), and the factor log2(e) goes into the exponent's FMA (mul). A masked key
+            // (past the row's bound, or a zero bit of a partial block) becomes -inf, in the
+            // chunks where some row of the warp has one.
+            mul = kLog2e;
+            const float scl = P.scale;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int lim = nvalid - 32 * c;
+              uint32_t keep = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
+              if constexpr (kMask == kMaskBits) keep &= bw[c];
+              float bias32[32];
+#pragma unroll
+              for (int e = 0; e < 32; e += 8) {
+                const int col = c * 32 + e;
+                float* f8 = bias32 + e;
+                if constexpr (kBias == kBiasTile) {
+                  // 128-byte swizzled rows: 16-byte chunk ch of row r sits at chunk ch ^ (r % 8)
+                  const int box = col >> 6, ch = (col & 63) >> 3;
+                  load8<BT>(reinterpret_cast<const BT*>(bsm + box * kRegionBytes + r * 128 + ((ch ^ (r & 7)) << 4)),
+                            *reinterpret_cast<float(*)[8]>(f8));
+                } else if (col + 8 <= nvalid) {
+                  load8<BT>(bias_row + key0 + col, *reinterpret_cast<float(*)[8]>(f8));
+                } else {
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) f8[k] = (col + k < nvalid) ? to_f32(bias_row[key0 + col + k]) : 0.f;
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float t0, t1;
+                fma2(t0, t1, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), scl, scl, bias32[e], bias32[e + 1]);
+                v[c][e] = __float_as_uint(t0);
+                v[c][e + 1] = __float_as_uint(t1);
+              }
+              if (__any_sync(0xffffffffu, keep != 0xffffffffu)) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[c][e] = ((keep >> e) & 1u) ? v[c][e] : 0xff800000u;
+              }
+#pragma unroll
+              for (int e = 0; e < 32; e += 2)
+                mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
+            }
           } else {
             mul = 1.f;
 #pragma unroll
@@ -993,31 +1026,28 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           if (P.lse && i < P.Lq)
             P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = (!pad && l > 0.f) ? m_used + log2f(l) : INFINITY;
         }
-        // O read out of TMEM in one batch (one wait), after which its columns are released to
-        // the next unit's first PV before the conversion and the stores
-        uint32_t o[D / 32][32];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_addr + ocol + c * 32, o[c]);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free[s]);
-        if (i < w.q_rows && row_ok) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + ocol + c * 32, o);
+          tmem_wait_ld();
+          if (i < w.q_rows && row_ok) {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint32_t wv[4];
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[c][e + 2 * k]) * inv : inv);
-                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[c][e + 2 * k + 1]) * inv : inv);
+                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k]) * inv : inv);
+                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[e + 2 * k + 1]) * inv : inv);
                 wv[k] = std::is_same<T, __half>::value ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
               }
               *reinterpret_cast<uint4*>(orow + c * 32 + e) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[s]);
       }
     }();
   }

@@ -103,12 +103,12 @@ cudaError_t launch_t(const void* x, void* out, long long rows, int nheads, int d
   return cudaGetLastError();
 }
 
-// cos / sin of every (row, pair c) angle, interleaved: table[(row * (d/2) + c) * 2 + {0, 1}],
-// the angle formed and reduced as in rope_kernel. The prefill kernel reads it to rotate its Q
-// tiles in shared memory.
+// (cos, sin) of every (row, pair c) angle as an fp16 pair, table[row * (d/2) + c], the angle
+// formed and reduced as in rope_kernel. The prefill kernel reads it to rotate its Q tiles in
+// shared memory (fp16 keeps 11 significant bits, finer than the bf16 of the rotated values).
 __global__ void __launch_bounds__(kThreads)
 rope_table_kernel(long long rows, int d, const int32_t* __restrict__ positions, double log2_base,
-                  float2* __restrict__ table) {
+                  __half2* __restrict__ table) {
   extern __shared__ double freq[];  // [d / 2]
   const int half = d / 2;
   for (int c = threadIdx.x; c < half; c += blockDim.x) freq[c] = exp2(-2.0 * (double)c / (double)d * log2_base);
@@ -123,7 +123,7 @@ rope_table_kernel(long long rows, int d, const int32_t* __restrict__ positions, 
     const double r = a - kTwoPi * rint(a / kTwoPi);
     float sn, cs;
     sincosf((float)r, &sn, &cs);
-    table[idx] = make_float2(cs, sn);
+    table[idx] = __floats2half2_rn(cs, sn);
   }
 }
 
@@ -139,7 +139,7 @@ cudaError_t launch_rope_table(long long rows, int d, const int32_t* positions, d
   const long long blocks = (rows * half + kThreads - 1) / kThreads;
   const unsigned grid = (unsigned)(blocks < 8LL * sms ? blocks : 8LL * sms);
   rope_table_kernel<<<grid, kThreads, sizeof(double) * half, stream>>>(rows, d, positions, log2(base),
-                                                                       static_cast<float2*>(table));
+                                                                       static_cast<__half2*>(table));
   return cudaGetLastError();
 }
 

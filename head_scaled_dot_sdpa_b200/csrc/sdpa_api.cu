@@ -333,7 +333,7 @@ RopeLayout rope_layout(const sdpa::Problem& P) {
   const size_t es = P.dtype == SDPA_F32 ? 4 : 2;
   L.k_off = kStatusBytes;
   L.table_off = L.k_off + round256((size_t)P.B * P.Lk * P.Hkv * P.D * es);
-  L.q_off = L.table_off + round256((size_t)P.B * P.Lq * (P.D / 2) * 2 * sizeof(float));
+  L.q_off = L.table_off + round256((size_t)P.B * P.Lq * (P.D / 2) * sizeof(uint32_t));
   L.total = L.q_off + round256((size_t)P.B * P.Lq * P.H * P.D * es) +
             round256(sdpa::prefill_workspace_bytes(P));
   return L;
@@ -373,7 +373,7 @@ sdpa_status sdpa_forward_rope(const sdpa_params* p, const int32_t* q_positions, 
     void* table = base_ws + L.table_off;
     e = sdpa::launch_rope_table((long long)P.B * P.Lq, P.D, q_positions, base, table, s);
     if (e != cudaSuccess) return cuda_fail(e, "rotary table");
-    P.q_rope = static_cast<const float2*>(table);
+    P.q_rope = static_cast<const uint32_t*>(table);
     const char* msg = nullptr;
     e = sdpa::launch_prefill(P, q, k_rot, v, out, base_ws + L.q_off, s, &msg);
     if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");

@@ -210,33 +210,6 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 2^x for a pair of finite x <= 128 on the FMA pipe, packed f32x2 (for moving part of a
-// row's exponentials off the MUFU unit). x = k + f with k = round(x) (added to the exponent
-// field) and f in [-1/2, 1/2], where a cubic fitted by the Remez exchange to 2^f (minimax in
-// relative error, 7.5e-5) gives the mantissa. Inputs below -126 are clamped there (2^-126,
-// which a 16-bit P rounds to 0 in fp16 and to a negligible value in bf16).
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  float t0, t1, k0, k1, f0, f1, p0, p1;
-  // t = x + 1.5 * 2^23 rounds x to the nearest integer in t's low mantissa bits
-  asm("{\n .reg .b64 rx, rm, rt;\n mov.b64 rx, {%2, %3};\n mov.b64 rm, {%4, %4};\n"
-      " add.rn.f32x2 rt, rx, rm;\n mov.b64 {%0, %1}, rt;\n}\n"
-      : "=f"(t0), "=f"(t1) : "f"(x0), "f"(x1), "f"(12582912.f));
-  asm("{\n .reg .b64 rt, rm, rk;\n mov.b64 rt, {%2, %3};\n mov.b64 rm, {%4, %4};\n"
-      " sub.rn.f32x2 rk, rt, rm;\n mov.b64 {%0, %1}, rk;\n}\n"
-      : "=f"(k0), "=f"(k1) : "f"(t0), "f"(t1), "f"(12582912.f));
-  asm("{\n .reg .b64 rx, rk, rf;\n mov.b64 rx, {%2, %3};\n mov.b64 rk, {%4, %5};\n"
-      " sub.rn.f32x2 rf, rx, rk;\n mov.b64 {%0, %1}, rf;\n}\n"
-      : "=f"(f0), "=f"(f1) : "f"(x0), "f"(x1), "f"(k0), "f"(k1));
-  fma2(p0, p1, 0.0551716691f, 0.0551716691f, f0, f1, 0.2426111222f, 0.2426111222f);
-  fma2(p0, p1, p0, p1, f0, f1, 0.6932609855f, 0.6932609855f);
-  fma2(p0, p1, p0, p1, f0, f1, 0.9999280735f, 0.9999280735f);
-  // k is in t's low mantissa bits (two's complement): shifted into the exponent field and added
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // max(a, b, c) in one instruction (three-input form of max.f32 on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
