@@ -113,6 +113,15 @@ bool backward_mma_supported(const Problem& P, const void* q, const void* k, cons
 cudaError_t launch_backward_mma(const Problem& P, const void* q, const void* k, const void* v, const void* out,
                                 const void* dout, void* dq, void* dk, void* dv, float* dscale, void* ws,
                                 cudaStream_t stream);
+// The same on the tcgen05 tensor cores (bf16 / fp16, head_dim = v_head_dim = 128, no bias, mask,
+// block info or packed sequences): delta, dK / dV per key tile, dQ / dscale per query tile.
+// lse and delta are [B][H][Lq] floats; lse (log2 units) must already hold the forward's row
+// log-sum-exp.
+bool backward_sm100_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out,
+                              const void* dout, const void* dq, const void* dk, const void* dv);
+cudaError_t launch_backward_sm100(const Problem& P, const void* q, const void* k, const void* v, const void* out,
+                                  const void* dout, void* dq, void* dk, void* dv, float* dscale, float* lse,
+                                  float* delta, cudaStream_t stream);
 // scaled_dot_product_attention_with_weights with dropout: mma.sync tiles (bf16 / fp16,
 // head_dim = v_head_dim = 64 or 128) or SIMT. Needs no workspace.
 bool weights_mma_supported(const Problem& P, const void* q, const void* k, const void* v, const void* out);

@@ -3,9 +3,9 @@
 #include <algorithm>
 
 #include "prefill_sm100.cuh"
+#include "tma_map.h"
 
 namespace sdpa {
-namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
@@ -39,6 +39,8 @@ bool make_map(CUtensorMap* m, const void* base, int dtype, int D, int heads, int
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 // The 16-bit bias as a 4-d tensor map (keys, queries, heads, batch) for the shared-memory bias
 // tiles: box = 64 keys x 128 queries, 128B swizzle. A broadcast head / batch dimension
@@ -159,6 +161,18 @@ cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const
   const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
   const int grid = (int)std::min<long long>(n_units, sm_count());
   cudaError_t e;
+  if (P.lse || P.q_rope) {
+    // the forward with its row log-sum-exp and / or rotated Q tiles (no bias or mask: checked by
+    // the callers)
+    if (P.dtype == SDPA_BF16)
+      e = P.D == 128 ? prefill::launch_aux<__nv_bfloat16, 128>(maps, P, out, grid, stream)
+                     : prefill::launch_aux<__nv_bfloat16, 64>(maps, P, out, grid, stream);
+    else
+      e = P.D == 128 ? prefill::launch_aux<__half, 128>(maps, P, out, grid, stream)
+                     : prefill::launch_aux<__half, 64>(maps, P, out, grid, stream);
+    if (e != cudaSuccess && msg) *msg = "prefill launch";
+    return e;
+  }
   if (P.dtype == SDPA_BF16)
     e = P.D == 128 ? prefill::launch<__nv_bfloat16, 128>(maps, P, out, grid, false, stream)
                    : prefill::launch<__nv_bfloat16, 64>(maps, P, out, grid, bias_tiles, stream);

@@ -72,10 +72,12 @@ constexpr int kSchedWord = 16;       // int offset in the status area of the uni
 // and key tile (head_dim 64, where the shared memory holds it); the others read global memory.
 enum { kBiasNone = 0, kBiasSame = 1, kBiasF32 = 2, kBiasTile = 3 };
 enum { kMaskNone = 0, kMaskDense = 1, kMaskBits = 2 };
-// kModeForward: the attention output (and, when P.lse is set, each row's log-sum-exp);
+// kModeForward: the attention output. kModeAux: the same, and (no bias or mask) each row's
+// log-sum-exp when P.lse is set and the rotary embedding of the Q tiles when P.q_rope is set.
 // kModeWeights: scaled_dot_product_attention_with_weights given that log-sum-exp: the exact
 // weights 2^(x - lse) of the visited key tiles, dropped out and stored, and out = sum w' v.
-enum { kModeForward = 0, kModeWeights = 2 };
+// (The plain forward carries none of the extra code.)
+enum { kModeForward = 0, kModeAux = 1, kModeWeights = 2 };
 
 // Shared-memory plan: the Q tiles of the two query tiles, the K and V rings, and with bias
 // tiles (kBT, head_dim 64) one bias tile per query tile. (A third Q slot, so that the next
@@ -579,7 +581,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         const uint32_t qtile = q_base + qslot * C::kTileBytes;
         if (my_n > 0) {
           // the Q tile loaded (and, with the rotary embedding, rotated in place)
-          if (!wait_all(P.q_rope ? &q_rot[qslot] : &q_full[qslot], (my_qi / C::kQSlots) & 1)) return;
+          if (!wait_all((kMode == kModeAux && P.q_rope) ? &q_rot[qslot] : &q_full[qslot], (my_qi / C::kQSlots) & 1))
+            return;
         }
         // V(x) loaded and, for the unit's first PV, O free: waited for ahead of the turn, so
         // that they are off the path from "P ready" to the MMA issue
@@ -707,7 +710,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         const QTile qt = s ? w.t[1] : w.t[0];
         const uint32_t my_qi = qi + ((s == 1 && w.t[0].n > 0) ? 1u : 0u);
         qi += (w.t[0].n > 0 ? 1u : 0u) + (w.t[1].n > 0 ? 1u : 0u);
-        if (P.q_rope && qt.n > 0) {
+        if (kMode == kModeAux && P.q_rope && qt.n > 0) {
           // Rotary embedding of this thread's query row in the tile's Q slot, once the tile
           // has landed: the pair (c, c + D/2) by the angle whose (cos, sin) the table holds
           // as fp16 for row b * Lq + i. 128-byte swizzle: logical 16-byte chunk x of row r
@@ -1021,7 +1024,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         tc_fence_after();
         const bool pad = i >= w.q_len;
         const float inv = (l > 0.f) ? 1.f / l : __int_as_float(0x7fc00000);
-        if constexpr (kMode == kModeForward) {
+        if constexpr (kMode == kModeAux) {
           // the row's log-sum-exp in log2 units, for a weights pass that follows
           if (P.lse && i < P.Lq)
             P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = (!pad && l > 0.f) ? m_used + log2f(l) : INFINITY;
@@ -1089,6 +1092,14 @@ template <> cudaError_t launch<__half, 64>(const TensorMaps&, const Problem&, vo
 // written P.lse and weights_fill_kernel the key tiles the pass does not visit.
 template <typename T, int D>
 cudaError_t launch_weights(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream);
+// The forward with the row log-sum-exp (P.lse) and / or the rotated Q tiles (P.q_rope); no bias
+// or mask.
+template <typename T, int D>
+cudaError_t launch_aux(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream);
+template <> cudaError_t launch_aux<__nv_bfloat16, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_aux<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_aux<__half, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_aux<__half, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
 template <> cudaError_t launch_weights<__nv_bfloat16, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
 template <> cudaError_t launch_weights<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
 template <> cudaError_t launch_weights<__half, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
@@ -1156,6 +1167,11 @@ inline int mask_variant(const Problem& P) {
 }
 
 #define SDPA_PREFILL_DEFINE_LAUNCH(T, D)                                                              \
+  template <>                                                                                       \
+  cudaError_t launch_aux<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,      \
+                               cudaStream_t stream) {                                               \
+    return launch_variant<T, D, kBiasNone, kMaskNone, kModeAux>(maps, P, out, grid, stream);       \
+  }                                                                                                 \
   template <>                                                                                       \
   cudaError_t launch_weights<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,  \
                                    cudaStream_t stream) {                                           \

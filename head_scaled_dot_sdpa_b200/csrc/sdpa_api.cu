@@ -368,7 +368,8 @@ sdpa_status sdpa_forward_rope(const sdpa_params* p, const int32_t* q_positions, 
   // the keys, rotated once: every query tile of the key/value head reads them
   cudaError_t e = sdpa::launch_rope(P.dtype, k, k_rot, (long long)P.B * P.Lk, P.Hkv, P.D, k_positions, base, s);
   if (e != cudaSuccess) return cuda_fail(e, "rotary embedding of the keys");
-  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && sdpa::prefill_supported(P, q, k_rot, v, out)) {
+  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && !P.bias && !P.mask && !P.bcls &&
+      sdpa::prefill_supported(P, q, k_rot, v, out)) {
     // the queries are rotated tile by tile in shared memory, from a cos / sin table
     void* table = base_ws + L.table_off;
     e = sdpa::launch_rope_table((long long)P.B * P.Lq, P.D, q_positions, base, table, s);
@@ -383,6 +384,14 @@ sdpa_status sdpa_forward_rope(const sdpa_params* p, const int32_t* q_positions, 
   void* q_rot = base_ws + L.q_off;
   e = sdpa::launch_rope(P.dtype, q, q_rot, (long long)P.B * P.Lq, P.H, P.D, q_positions, base, s);
   if (e != cudaSuccess) return cuda_fail(e, "rotary embedding of the queries");
+  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && sdpa::prefill_supported(P, q_rot, k_rot, v, out)) {
+    // a bias or a mask: the queries rotated into the workspace, then the tcgen05 forward
+    const char* msg = nullptr;
+    e = sdpa::launch_prefill(P, q_rot, k_rot, v, out, nullptr, s, &msg);
+    if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");
+    g_last_kernel = "prefill_tcgen05";
+    return SDPA_OK;
+  }
   if (!generic_ok(P))
     return fail(SDPA_ERR_UNSUPPORTED, "head sizes dqk=%d dv=%d exceed the SIMT kernel's limits (1024, 256)",
                 P.D, P.Dv);
@@ -416,6 +425,22 @@ sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, co
     return fail(SDPA_ERR_INVALID_ARG, "q, k, v, out, dout, dq, dk and dv must not be NULL");
   P.status = static_cast<int*>(ws);
   void* scratch = static_cast<char*>(ws) + kStatusBytes;
+  if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && sdpa::backward_sm100_supported(P, q, k, v, out, dout, dq, dk, dv) &&
+      sdpa::prefill_supported(P, q, k, v, dq)) {
+    // tcgen05: the forward again, for the row log-sum-exp (its output goes to dq, which the
+    // gradient overwrites), then delta, dK / dV and dQ / dscale
+    float* lse = static_cast<float*>(scratch);
+    float* delta = lse + (size_t)P.B * P.H * P.Lq;
+    sdpa::Problem F = P;
+    F.lse = lse;
+    const char* msg = nullptr;
+    cudaError_t e = sdpa::launch_prefill(F, q, k, v, dq, nullptr, (cudaStream_t)stream, &msg);
+    if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");
+    e = sdpa::launch_backward_sm100(P, q, k, v, out, dout, dq, dk, dv, dscale, lse, delta, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gradient launch");
+    g_last_kernel = "backward_tcgen05";
+    return SDPA_OK;
+  }
   if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && sdpa::backward_mma_supported(P, q, k, v, out, dout)) {
     cudaError_t e = sdpa::launch_backward_mma(P, q, k, v, out, dout, dq, dk, dv, dscale, scratch, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "gradient launch");

@@ -256,10 +256,11 @@ SDPA_API sdpa_status sdpa_rope(const void* x, void* out, sdpa_dtype dtype, int64
  *  - The workspace (sdpa_rope_workspace_size(p) bytes) holds the status word, the rotated keys
  *    (one pass over k: every query tile of a key/value head reads them), a cos / sin table of
  *    the query rows and room for rotated queries.
- *  - Kernels. Where sdpa_forward takes the tcgen05 kernel, a table kernel computes the query
- *    angles' cos / sin and the attention kernel rotates each Q tile in shared memory after
- *    its TMA load, before the first QK^T MMA reads it, so the rotated queries never go to
- *    memory. Otherwise the queries are rotated into the workspace and the SIMT kernel runs.
+ *  - Kernels. Where sdpa_forward takes the tcgen05 kernel and there is no bias or mask, a table
+ *    kernel computes the query angles' cos / sin and the attention kernel rotates each Q tile
+ *    in shared memory after its TMA load, before the first QK^T MMA reads it, so the rotated
+ *    queries never go to memory. Otherwise the queries are rotated into the workspace and the
+ *    tcgen05 kernel (with a bias or mask) or the SIMT kernel runs.
  *    The rotated values are rounded to the input type, as sdpa_rope's output is. */
 SDPA_API size_t sdpa_rope_workspace_size(const sdpa_params* p);
 SDPA_API sdpa_status sdpa_forward_rope(const sdpa_params* p, const int32_t* q_positions,

@@ -41,10 +41,13 @@ def _inputs(seed, B, Lq, Lk, H, Hkv, D, Dv, dtype):
             si.normal(rng, (B, Lk, Hkv, Dv), n), si.normal(rng, (B, Lq, H, Dv), n))
 
 
-def expected_kernel(q, v, generic=False):
-    """mma.sync tiles for 16-bit types with head_dim = v_head_dim = 64 or 128, SIMT otherwise."""
+def expected_kernel(q, v, generic=False, masked=False):
+    """16-bit types: head_dim = v_head_dim = 128 without a mask on tcgen05, 64 or 128 on mma.sync
+    tiles; SIMT otherwise."""
     tiles = q.dtype in (torch.bfloat16, torch.float16) and q.shape[-1] == v.shape[-1] in (64, 128)
-    return "backward_mma" if tiles and not generic else "backward_simt"
+    if generic or not tiles:
+        return "backward_simt"
+    return "backward_tcgen05" if q.shape[-1] == 128 and not masked else "backward_mma"
 
 
 def check(q, k, v, dout, what, generic=False, **kw):
@@ -53,7 +56,7 @@ def check(q, k, v, dout, what, generic=False, **kw):
     qd, kd, vd, dd = (t.to(DEV) for t in (q, k, v, dout))
     out = sdpa.sdpa_forward(qd, kd, vd, **kw)
     dq, dk, dv, ds = sdpa.sdpa_backward(qd, kd, vd, out, dd, generic=generic, **kw)
-    assert sdpa.last_kernel() == expected_kernel(q, v, generic)
+    assert sdpa.last_kernel() == expected_kernel(q, v, generic, masked="mask" in kw or "block_info" in kw)
     assert sdpa.read_device_status() == sdpa.SDPA_OK
     okw = {a: b for a, b in kw.items() if a != "block_info"}
     if "mask" in okw:
@@ -90,6 +93,15 @@ def test_backward_shapes(dtype, shape, causal):
     check(q, k, v, dout, f"{shape} causal={causal}", is_causal=causal)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("causal", [False, True, "bottom_right"])
+def test_backward_tcgen05_gqa_tiles(dtype, causal):
+    """The tcgen05 gradient with several query and key tiles per unit, ragged tails on both,
+    unequal lengths and GQA groups of 4."""
+    q, k, v, dout = _inputs(31, 2, 300, 389, 8, 2, 128, 128, dtype)
+    check(q, k, v, dout, f"tcgen05 gqa causal={causal}", is_causal=causal)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_backward_simt_forced(causal):
     """The SIMT kernels on a shape the tiles also take, so both paths stay covered."""
@@ -104,6 +116,10 @@ def test_backward_lengths_offsets_and_empty_rows(dtype):
     q, k, v, dout = _inputs(5, 3, 50, 70, 4, 2, 64, 64, dtype)
     check(q, k, v, dout, "lengths", is_causal=True, q_offset=[20, -5, 0], q_lengths=[50, 31, 12],
           kv_lengths=[70, 40, 0])
+    if dtype != torch.float32:  # the same on the tcgen05 kernels (head_dim 128), tiles ragged
+        q, k, v, dout = _inputs(7, 3, 200, 270, 4, 2, 128, 128, dtype)
+        check(q, k, v, dout, "lengths tcgen05", is_causal=True, q_offset=[20, -5, 0], q_lengths=[200, 131, 12],
+              kv_lengths=[270, 140, 0])
 
 
 def test_backward_mask_and_block_info():
@@ -127,6 +143,7 @@ def test_backward_full_size_sampled():
     qd, kd, vd, dd = (t.to(DEV) for t in (q, k, v, dout))
     out = sdpa.sdpa_forward(qd, kd, vd, is_causal=True)
     dq, dk, dv, _ = sdpa.sdpa_backward(qd, kd, vd, out, dd, is_causal=True)
+    assert sdpa.last_kernel() == "backward_tcgen05"
     assert sdpa.read_device_status() == sdpa.SDPA_OK
     dq, dk, dv = dq.cpu(), dk.cpu(), dv.cpu()
     g = w.nheads // w.nkvheads

@@ -143,3 +143,20 @@ def test_sliding_window_chunked_prefill():
     mask[..., P - W:] = True
     want = oracle.sdpa_forward(f64(qr[:, P:]), f64(kr), f64(v), mask=mask, is_causal=True, q_offset=P)
     assert_matches(out, want, 1e-2, "sliding-window chunk")
+
+
+def test_fused_rope_with_a_mask_rotates_into_the_workspace():
+    """With a mask the queries are rotated into the workspace and the tcgen05 kernel takes the
+    rotated arrays with its dense-mask variant."""
+    rng = np.random.Generator(np.random.PCG64(78))
+    B, Lq, Lk, H, Hkv, D = 1, 160, 192, 4, 2, 128
+    q, k, v = (si.normal(rng, s, "bf16") for s in [(B, Lq, H, D), (B, Lk, Hkv, D), (B, Lk, Hkv, D)])
+    qpos, kpos = rng.integers(0, 9000, size=B * Lq).astype(np.int32), rng.integers(0, 9000, size=B * Lk).astype(np.int32)
+    mask = torch.from_numpy(rng.random((H, Lq, Lk)) < 0.7)
+    out = sdpa.sdpa_forward_rope(q.to(DEV), k.to(DEV), v.to(DEV), torch.from_numpy(qpos), torch.from_numpy(kpos),
+                                 mask=mask.to(DEV))
+    assert sdpa.last_kernel() == "prefill_tcgen05"
+    qr = _rounded(oracle.rope(f64(q).reshape(Lq, H, D), qpos), torch.bfloat16).reshape(B, Lq, H, D)
+    kr = _rounded(oracle.rope(f64(k).reshape(Lk, Hkv, D), kpos), torch.bfloat16).reshape(B, Lk, Hkv, D)
+    want = oracle.sdpa_forward(qr, kr, f64(v), mask=mask.numpy()[None])
+    assert_matches(out, want, 1e-2, "rope + mask")
