@@ -396,18 +396,20 @@ def packed_workload(args, dev, world, ws, peaks):
 
 
 def backward_workload(args, dev, world, ws, peaks):
-    """The fused gradient (dq, dk, dv, dscale) of the causal GQA prefill workload: 10*head_dim
-    flops per attended pair (the logits recomputed, dout.v, and the dv, dq and dk products;
-    the tiled kernels also recompute the logits once more for the row log-sum-exp, which is
-    not counted)."""
+    """The fused gradient (dq, dk, dv, dscale) of the causal GQA prefill workload, given the row
+    log-sum-exp the forward kept (sdpa_forward_lse, outside the timed region, as in a training
+    step): 10*head_dim flops per attended pair (the logits recomputed, dout.v, and the dv, dq
+    and dk products; the recomputation of the logits in both gradient kernels and the low parts
+    of dx are not counted). Three launches: delta, dK/dV, dQ."""
     import head_scaled_dot_sdpa_b200 as sdpa
 
     w = si.CAUSAL_GQA_PREFILL
     q, k, v = [t.to(dev) for t in si.qkv(w)]
     dout = si.normal(si.rng_for(w.seed + 7), tuple(q.shape), w.dtype).to(dev)
-    out = sdpa.sdpa_forward(q, k, v, is_causal=True, workspace=ws)
+    # the forward of the training step keeps the row log-sum-exp for the gradient
+    out, lse = sdpa.sdpa_forward_lse(q, k, v, is_causal=True, workspace=ws)
     flops = 10.0 * w.head_dim * w.batch * w.nheads * causal_pairs(w.q_len, w.kv_len)
-    step = lambda: sdpa.sdpa_backward(q, k, v, out, dout, is_causal=True, workspace=ws)
+    step = lambda: sdpa.sdpa_backward(q, k, v, out, dout, is_causal=True, lse=lse, workspace=ws)
     per = time_steps(step, max(3, args.steps // 4), args.warmup, world)
     ms = max_over_ranks(float(np.mean(per)), world)
     tf = flops / (ms * 1e-3) / 1e12
@@ -415,7 +417,8 @@ def backward_workload(args, dev, world, ws, peaks):
             "ms_per_step": round(ms, 3), "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
                          "frac": round(tf / peaks["bf16"], 5)},
-            "kernel": sdpa.last_kernel(), "gpu_launches_per_step": 2 if sdpa.last_kernel() == "backward_mma" else 3}
+            "kernel": sdpa.last_kernel(),
+            "gpu_launches_per_step": {"backward_tcgen05": 3, "backward_mma": 2}.get(sdpa.last_kernel(), 3)}
 
 
 def weights_workload(args, dev, world, ws, peaks):

@@ -94,6 +94,8 @@ _lib.sdpa_rope_workspace_size.argtypes = [_PP]
 _lib.sdpa_rope_workspace_size.restype = _sz
 _lib.sdpa_forward_rope.argtypes = [_PP, _vp, _vp, ctypes.c_double, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sdpa_backward.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sdpa_backward_lse.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sdpa_forward_lse.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sdpa_decode_with_cache.argtypes = [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.cache_update_at_index.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32,
                                        _i32, _vp, _vp, _vp]
@@ -358,13 +360,36 @@ def sdpa_rope(x, positions, base=10000.0, *, out=None, stream=None):
     return out
 
 
+def sdpa_forward_lse(q, k, v, *, scale=None, is_causal=False, q_offset=0, q_lengths=None, kv_lengths=None,
+                     out=None, workspace=None, stream=None):
+    """sdpa_forward that also returns each query row's log-sum-exp (natural log, (B, H, Lq)
+    float32; +inf for rows with no key or past q_lengths), for sdpa_backward(lse=...). The
+    tcgen05 kernel only: bf16/fp16, head sizes 64 or 128, no bias or mask."""
+    _check_qkv(q, k, v)
+    keep = []
+    p = _params(q, k, v, bias=None, mask=None, scale=scale, is_causal=is_causal, q_offset=q_offset,
+                q_lengths=q_lengths, kv_lengths=kv_lengths, block_info=None, flags=0, keep=keep)
+    if out is None:
+        out = torch.empty(q.shape[:3] + (v.shape[3],), dtype=q.dtype, device=q.device)
+    lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=q.device)
+    need = _lib.sdpa_workspace_size(ctypes.byref(p))
+    if need == 0:
+        raise SdpaError(SDPA_ERR_INVALID_ARG, _lib.sdpa_last_error().decode())
+    ws = _workspace(q.device, need, workspace)
+    _check(_lib.sdpa_forward_lse(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), lse.data_ptr(), ws.ptr,
+                                 ws.nbytes, _stream(stream)))
+    return out, lse
+
+
 def sdpa_backward(q, k, v, out, dout, *, mask=None, scale=None, is_causal=False, q_offset=0,
-                  q_lengths=None, kv_lengths=None, block_info=None, workspace=None, generic=False,
+                  q_lengths=None, kv_lengths=None, block_info=None, lse=None, workspace=None, generic=False,
                   stream=None):
     """The gradient of the fused implementation for the loss sum(dout * out), where `out` is
     sdpa_forward(q, k, v; ...) with the same arguments: returns (dq, dk, dv, dscale), dscale a
     0-d float32 device tensor. Rows with no attended key and rows past q_lengths take no part.
-    No bias (the page's automatic differentiation takes the materialized implementation then)."""
+    No bias (the page's automatic differentiation takes the materialized implementation then).
+    lse: the row log-sum-exp sdpa_forward_lse returned for the same call (the tcgen05 gradient
+    then does not run the forward again)."""
     _check_qkv(q, k, v)
     for n, t in (("out", out), ("dout", dout)):
         if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype or t.shape != q.shape[:3] + (v.shape[3],):
@@ -379,8 +404,16 @@ def sdpa_backward(q, k, v, out, dout, *, mask=None, scale=None, is_causal=False,
     if need == 0:
         raise SdpaError(SDPA_ERR_INVALID_ARG, _lib.sdpa_last_error().decode())
     ws = _workspace(q.device, need, workspace)
-    _check(_lib.sdpa_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(dq),
-                              _ptr(dk), _ptr(dv), dscale.data_ptr(), ws.ptr, ws.nbytes, _stream(stream)))
+    if lse is None:
+        _check(_lib.sdpa_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), dscale.data_ptr(), ws.ptr, ws.nbytes, _stream(stream)))
+    else:
+        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous() or \
+                tuple(lse.shape) != (q.shape[0], q.shape[2], q.shape[1]):
+            raise ValueError("lse must be the contiguous float32 (B, H, Lq) CUDA tensor sdpa_forward_lse returned")
+        _check(_lib.sdpa_backward_lse(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
+                                      lse.data_ptr(), _ptr(dq), _ptr(dk), _ptr(dv), dscale.data_ptr(), ws.ptr,
+                                      ws.nbytes, _stream(stream)))
     return dq, dk, dv, dscale
 
 
@@ -538,6 +571,6 @@ def build_block_mask_info(mask, bq: int = 128, bk: int = 128, *, stream=None) ->
     return info
 
 
-__all__ = ["sdpa_forward", "sdpa_forward_packed", "sdpa_forward_rope", "sdpa_forward_with_weights", "sdpa_rope", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
+__all__ = ["sdpa_forward", "sdpa_forward_lse", "sdpa_forward_packed", "sdpa_forward_rope", "sdpa_forward_with_weights", "sdpa_rope", "sdpa_backward", "sdpa_decode_with_cache", "cache_update_at_index",
            "build_block_mask_info", "BlockMaskInfo", "Workspace", "read_device_status",
            "last_kernel", "SdpaError", "lib"]

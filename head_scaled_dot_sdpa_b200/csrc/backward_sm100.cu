@@ -24,7 +24,7 @@
 // the sum over a row cancels (sum_j dx_ij = 0). w >= 0 enters dV with one rounding (its sum
 // does not cancel: a relative error near 2^-9 / sqrt(3)).
 // TMEM columns (512): bwd_kv: S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512);
-// bwd_q: S [0,128), dP [128,256), dQ [256,384). A 32-column chunk of S (or dP) receives, once
+// bwd_q: S [0,128) and [384,512) (alternate key tiles), dP [128,256), dQ [256,384). A 32-column chunk of S (or dP) receives, once
 // read, the high parts of its 32 values (16 columns of 16-bit pairs) then the low parts (w^T:
 // the high parts only).
 // Warp roles (384 threads): warps 0-7 elementwise (warp w: TMEM lanes 32 (w % 4).., value
@@ -234,8 +234,10 @@ bwd_kv_kernel(const __grid_constant__ Maps maps, const Problem P, const float* _
   uint64_t* kv_empty = bars + 1;
   uint64_t* qd_full = bars + 2;   // [2]
   uint64_t* qd_empty = bars + 4;  // [2]
-  uint64_t* st_full = bars + 6;
-  uint64_t* pt_full = bars + 7;
+  uint64_t* st_full = bars + 6;    // S^T of the step computed
+  uint64_t* pt_full = bars + 7;    // w^T of the step written back (dV may start)
+  uint64_t* dp_full = bars + 22;   // dP^T of the step computed
+  uint64_t* dx_full = bars + 23;   // dx^T of the step written back (dK may start)
   uint64_t* acc_full = bars + 8;
   uint64_t* acc_free = bars + 9;
   uint64_t* drain = bars + 10;
@@ -257,6 +259,8 @@ bwd_kv_kernel(const __grid_constant__ Maps maps, const Problem P, const float* _
     }
     mbar_init(st_full, 1);
     mbar_init(pt_full, kEw);
+    mbar_init(dp_full, 1);
+    mbar_init(dx_full, kEw);
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kEw);
     mbar_init(drain, 1);
@@ -352,23 +356,43 @@ bwd_kv_kernel(const __grid_constant__ Maps maps, const Problem P, const float* _
         if (qe <= qb) continue;
         if (!W.all(kv_full, uc & 1)) return;
         const int steps = P.group * (qe - qb);
+        // Issue order per step n: dV(n), S^T(n+1), dK(n), dP^T(n+1). The elementwise warps
+        // publish w^T(n) before they read dP^T(n), so the exponentials of step n+1 run while
+        // dK(n) and dP^T(n+1) are on the tensor pipe. S^T(n+1) overwrites w^T(n) after dV(n)
+        // has read it, dP^T(n+1) overwrites dx^T(n) after dK(n): the pipe runs in order.
+        if (!W.all(&qd_full[n & 1], (n >> 1) & 1)) return;
+        tc_fence_after();
+        if (elected) {
+          mma_kmajor(st_t, k_a, q_a + (n & 1) * kTile, idesc_s);    // S^T = K Q^T
+          mma_commit(st_full);
+          mma_kmajor(dp_t, v_a, do_a + (n & 1) * kTile, idesc_s);   // dP^T = V dout^T
+          mma_commit(dp_full);
+        }
+        __syncwarp();
         for (int s = 0; s < steps; ++s, ++n) {
-          const int slot = n & 1;
-          if (!W.all(&qd_full[slot], (n >> 1) & 1)) return;
-          tc_fence_after();
-          if (elected) {
-            mma_kmajor(st_t, k_a, q_a + slot * kTile, idesc_s);    // S^T = K Q^T
-            mma_kmajor(dp_t, v_a, do_a + slot * kTile, idesc_s);   // dP^T = V dout^T
-            mma_commit(st_full);
-          }
-          __syncwarp();
+          const int slot = n & 1, nslot = (n + 1) & 1;
+          const bool more = s + 1 < steps;
           if (!W.all(pt_full, n & 1)) return;
           if (s == 0 && !W.all(acc_free, (uc & 1) ^ 1)) return;
+          if (more && !W.all(&qd_full[nslot], ((n + 1) >> 1) & 1)) return;
           tc_fence_after();
           if (elected) {
             mma_tmem_a(dv_t, st_t, do_a + slot * kTile, idesc_acc, s > 0, 1);  // dV += w^T dout
-            mma_tmem_a(dk_t, dp_t, q_a + slot * kTile, idesc_acc, s > 0);   // dK += dx^T Q
+            if (more) {
+              mma_kmajor(st_t, k_a, q_a + nslot * kTile, idesc_s);
+              mma_commit(st_full);
+            }
+          }
+          __syncwarp();
+          if (!W.all(dx_full, n & 1)) return;
+          tc_fence_after();
+          if (elected) {
+            mma_tmem_a(dk_t, dp_t, q_a + slot * kTile, idesc_acc, s > 0);  // dK += dx^T Q
             mma_commit(&qd_empty[slot]);
+            if (more) {
+              mma_kmajor(dp_t, v_a, do_a + nslot * kTile, idesc_s);
+              mma_commit(dp_full);
+            }
           }
           __syncwarp();
         }
@@ -418,7 +442,7 @@ bwd_kv_kernel(const __grid_constant__ Maps maps, const Problem P, const float* _
             const int i = qt * kBlk + (t & 127);
             const long long idx = ((long long)b * P.H + h) * P.Lq + i;
             float val = (t < 128) ? INFINITY : 0.f;
-            if (i < P.Lq) val = (t < 128) ? lse[idx] : delta[idx];
+            if (i < P.Lq) val = (t < 128) ? lse[idx] * P.lse_in_mul : delta[idx];
             st[t] = val;
           }
           // every warp's values are in (a step's slot is rewritten two steps later, after every
@@ -431,42 +455,68 @@ bwd_kv_kernel(const __grid_constant__ Maps maps, const Problem P, const float* _
           // key j attends queries [i_lo, i_hi): i < q_len, j < kv_len and (causal) j <= offset + i
           const int i_lo = P.causal != SDPA_CAUSAL_NONE ? j - bi.offset : 0;
           const int i_hi = j < bi.kv_len ? bi.q_len : 0;
-#pragma unroll 1
+          // phase 1: w^T from S^T, written back as 16-bit values (kept in fp32 for dx)
+          float wv[2][32];
+#pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             const int c = 2 * half + cc;  // 32-query chunk
             const int q0 = qt * kBlk + 32 * c;
             const uint32_t keep = range_bits(i_lo - q0, i_hi - q0);
-            uint32_t sv[32], dpv[32];
+            uint32_t sv[32];
             tmem_ld32(lane_addr + 32 * c, sv);
-            tmem_ld32(lane_addr + 128 + 32 * c, dpv);
             tmem_wait_ld();
             const float4* l4 = reinterpret_cast<const float4*>(st + 32 * c);
-            const float4* d4 = reinterpret_cast<const float4*>(st + kBlk + 32 * c);
-            uint32_t wo[16], xo[32];
+            uint32_t wo[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-              const float4 L = l4[e / 4], Dl = d4[e / 4];
-              const float lv[4] = {L.x, L.y, L.z, L.w}, dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
+              const float4 L = l4[e / 4];
+              const float lv[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
               for (int y = 0; y < 4; y += 2) {
                 const int f = e + y;
-                float x0, x1, t0, t1, d0, d1;
+                float x0, x1;
                 fma2(x0, x1, __uint_as_float(sv[f]), __uint_as_float(sv[f + 1]), sl2, sl2, -lv[y], -lv[y + 1]);
-                const float p0 = ((keep >> f) & 1u) ? ex2(x0) : 0.f;
-                const float p1 = ((keep >> (f + 1)) & 1u) ? ex2(x1) : 0.f;
-                wo[f / 2] = pack16<T>(p0, p1);
-                add2(t0, t1, __uint_as_float(dpv[f]), __uint_as_float(dpv[f + 1]), -dl[y], -dl[y + 1]);
-                fma2(d0, d1, p0, p1, t0, t1, 0.f, 0.f);  // dx = w (dp - delta)
-                split_pair<T>(d0, d1, xo[f / 2], xo[16 + f / 2]);
+                wv[cc][f] = ((keep >> f) & 1u) ? ex2(x0) : 0.f;
+                wv[cc][f + 1] = ((keep >> (f + 1)) & 1u) ? ex2(x1) : 0.f;
+                wo[f / 2] = pack16<T>(wv[cc][f], wv[cc][f + 1]);
               }
             }
             tmem_st16(lane_addr + 32 * c, wo);
-            tmem_st32(lane_addr + 128 + 32 * c, xo);
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (elected) mbar_arrive(pt_full);
+          // phase 2: dx^T = w^T (dP^T - delta), high and low parts over dP^T
+          if (!W.all(dp_full, n & 1)) return;
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
+            uint32_t dpv[32];
+            tmem_ld32(lane_addr + 128 + 32 * c, dpv);
+            tmem_wait_ld();
+            const float4* d4 = reinterpret_cast<const float4*>(st + kBlk + 32 * c);
+            uint32_t xo[32];
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 Dl = d4[e / 4];
+              const float dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
+#pragma unroll
+              for (int y = 0; y < 4; y += 2) {
+                const int f = e + y;
+                float t0, t1, d0, d1;
+                add2(t0, t1, __uint_as_float(dpv[f]), __uint_as_float(dpv[f + 1]), -dl[y], -dl[y + 1]);
+                fma2(d0, d1, wv[cc][f], wv[cc][f + 1], t0, t1, 0.f, 0.f);  // dx = w (dp - delta)
+                split_pair<T>(d0, d1, xo[f / 2], xo[16 + f / 2]);
+              }
+            }
+            tmem_st32(lane_addr + 128 + 32 * c, xo);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (elected) mbar_arrive(dx_full);
         }
         // epilogue: dK (warps 0-3, times scale) or dV (warps 4-7), one row per thread
         if (!W.all(acc_full, uc & 1)) return;
@@ -625,7 +675,8 @@ bwd_q_kernel(const __grid_constant__ Maps maps, const Problem P, const float* __
       constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
       constexpr uint32_t idesc_s = instr_desc_f16(kBf16, false, false, kBlk, kBlk);
       constexpr uint32_t idesc_acc = instr_desc_f16(kBf16, false, true, kBlk, kD);
-      const uint32_t s_t = tmem, dp_t = tmem + 128, dq_t = tmem + 256;
+      const uint32_t dp_t = tmem + 128, dq_t = tmem + 256;
+      auto s_tm = [&](uint32_t x) { return tmem + ((x & 1) ? 384u : 0u); };  // S, two buffers
       const uint32_t q_a = smem_addr(q_s), do_a = smem_addr(do_s), k_a = smem_addr(k_s), v_a = smem_addr(v_s);
       uint32_t uc = 0, n = 0;
       for (uint32_t kq = 0;; ++kq) {
@@ -638,21 +689,36 @@ bwd_q_kernel(const __grid_constant__ Maps maps, const Problem P, const float* __
         const int nk = kt_end_of(P, bi, qt);
         if (nk == 0) continue;
         if (!W.all(qo_full, uc & 1)) return;
+        // Issue order: S(0), dP(0); then per key tile kt (ring position n): S(n+1) into the other
+        // S buffer while the elementwise warps work on n, then (dx(n) written) dP(n+1) and
+        // dQ(n). The elementwise phase of n+1 then waits for dP(n+1) only, and runs while
+        // dQ(n) is on the tensor pipe. S(n+2) reuses the buffer of S(n) after dQ(n) read it.
+        if (!W.all(&kv_full[n & 1], (n >> 1) & 1)) return;
+        tc_fence_after();
+        if (elected) {
+          mma_kmajor(s_tm(n), q_a, k_a + (n & 1) * kTile, idesc_s);  // S = Q K^T
+          mma_kmajor(dp_t, do_a, v_a + (n & 1) * kTile, idesc_s);    // dP = dout V^T
+          mma_commit(s_full);
+        }
+        __syncwarp();
         for (int kt = 0; kt < nk; ++kt, ++n) {
-          const int slot = n & 1;
-          if (!W.all(&kv_full[slot], (n >> 1) & 1)) return;
-          tc_fence_after();
-          if (elected) {
-            mma_kmajor(s_t, q_a, k_a + slot * kTile, idesc_s);    // S = Q K^T
-            mma_kmajor(dp_t, do_a, v_a + slot * kTile, idesc_s);  // dP = dout V^T
-            mma_commit(s_full);
+          const int slot = n & 1, nslot = (n + 1) & 1;
+          const bool more = kt + 1 < nk;
+          if (more) {
+            if (!W.all(&kv_full[nslot], ((n + 1) >> 1) & 1)) return;
+            tc_fence_after();
+            if (elected) mma_kmajor(s_tm(n + 1), q_a, k_a + nslot * kTile, idesc_s);
+            __syncwarp();
           }
-          __syncwarp();
           if (!W.all(p_full, n & 1)) return;
           if (kt == 0 && !W.all(acc_free, (uc & 1) ^ 1)) return;
           tc_fence_after();
           if (elected) {
-            mma_tmem_a(dq_t, s_t, k_a + slot * kTile, idesc_acc, kt > 0);  // dQ += dx K
+            if (more) {
+              mma_kmajor(dp_t, do_a, v_a + nslot * kTile, idesc_s);
+              mma_commit(s_full);
+            }
+            mma_tmem_a(dq_t, s_tm(n), k_a + slot * kTile, idesc_acc, kt > 0);  // dQ += dx K
             mma_commit(&kv_empty[slot]);
           }
           __syncwarp();
@@ -692,7 +758,7 @@ bwd_q_kernel(const __grid_constant__ Maps maps, const Problem P, const float* __
           continue;
         }
         const long long ridx = ((long long)b * P.H + h) * P.Lq + i;
-        const float lse_i = i < P.Lq ? lse[ridx] : INFINITY;
+        const float lse_i = i < P.Lq ? lse[ridx] * P.lse_in_mul : INFINITY;
         const float delta_i = i < P.Lq ? delta[ridx] : 0.f;
         long long lim = i < bi.q_len ? bi.kv_len : 0;
         if (P.causal != SDPA_CAUSAL_NONE) lim = min(lim, (long long)bi.offset + i + 1);
@@ -705,7 +771,8 @@ bwd_q_kernel(const __grid_constant__ Maps maps, const Problem P, const float* __
             const int c = 2 * half + cc;  // 32-key chunk
             const uint32_t keep = range_bits(0, j_lim - (kt * kBlk + 32 * c));
             uint32_t sv[32], dpv[32];
-            tmem_ld32(lane_addr + 32 * c, sv);
+            const uint32_t scol = ((n & 1) ? 384u : 0u) + 32 * c;
+            tmem_ld32(lane_addr + scol, sv);
             tmem_ld32(lane_addr + 128 + 32 * c, dpv);
             tmem_wait_ld();
             uint32_t xo[32];
@@ -721,7 +788,7 @@ bwd_q_kernel(const __grid_constant__ Maps maps, const Problem P, const float* __
               fma2(ds_acc0, ds_acc1, d0, d1, s0, s1, ds_acc0, ds_acc1);
               split_pair<T>(d0, d1, xo[e / 2], xo[16 + e / 2]);
             }
-            tmem_st32(lane_addr + 32 * c, xo);
+            tmem_st32(lane_addr + scol, xo);
           }
           tmem_wait_st();
           tc_fence_before();

@@ -47,6 +47,8 @@ struct Problem {
   // the weights pass reads it, writes the weights [B][H][Lq][Lk] and applies the dropout
   // (keep when the row's 16-bit draw >= drop_thr, then scale by inv_keep)
   float* lse;
+  float lse_out_mul;  // the forward stores lse (log2 units) times this (ln 2: natural log); 1 by default
+  float lse_in_mul;   // the gradient reads lse times this as log2 units (log2 e for a natural log)
   void* weights;
   unsigned long long drop_seed;
   unsigned drop_thr;
@@ -71,6 +73,12 @@ struct BatchInfo {
 
 // Records the message sdpa_last_error() returns on this host thread.
 void set_last_error(const char* msg);
+
+// sdpa_backward (lse null: the forward runs again for the row log-sum-exp) and
+// sdpa_backward_lse (lse: the caller's, natural log, from sdpa_forward_lse).
+sdpa_status backward(const sdpa_params* p, const void* q, const void* k, const void* v, const void* out,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv, float* dscale, void* ws,
+                     size_t ws_bytes, cudaStream_t stream);
 
 // sdpa_decode_with_cache. Every argument is checked before anything is queued; with
 // clear_status the status word at the start of `ws` is then zeroed on `stream` before the

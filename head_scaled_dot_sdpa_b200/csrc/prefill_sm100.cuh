@@ -733,6 +733,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                                          (P.q_start ? (long long)P.Lq_total : (long long)P.B * P.Lq)));
         if (qt.n == 0) {
           // no key tile: NaN rows (nothing attended) or zero rows (past q_lengths)
+          if constexpr (kMode == kModeAux) {
+            if (P.lse && i < P.Lq) P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = INFINITY;
+          }
           if (i < w.q_rows && row_ok) {
             const float val = (i >= w.q_len) ? 0.f : __int_as_float(0x7fc00000);
             const uint32_t wv = std::is_same<T, __half>::value ? pack_f16x2(val, val) : pack_bf16x2(val, val);
@@ -1027,7 +1030,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if constexpr (kMode == kModeAux) {
           // the row's log-sum-exp in log2 units, for a weights pass that follows
           if (P.lse && i < P.Lq)
-            P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = (!pad && l > 0.f) ? m_used + log2f(l) : INFINITY;
+            P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] =
+                (!pad && l > 0.f) ? (m_used + log2f(l)) * P.lse_out_mul : INFINITY;
         }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {

@@ -95,6 +95,8 @@ sdpa_status resolve(const sdpa_params* p, sdpa::Problem* P) {
     P->ms[d] = p->mask_stride[d];
   }
   P->mask = p->mask;
+  P->lse_out_mul = 1.f;
+  P->lse_in_mul = 1.f;
   P->wait_timeout_ns = 1000000000ull;  // 1 s: far beyond any legitimate wait
   if (p->flags & SDPA_FLAG_SELFTEST_STALL) {
     P->wait_timeout_ns = 1000000ull;  // 1 ms
@@ -180,6 +182,30 @@ sdpa_status sdpa_forward(const sdpa_params* p, const void* q, const void* k, con
   cudaError_t e = sdpa::launch_generic(P, q, k, v, out, s);
   if (e != cudaSuccess) return cuda_fail(e, "generic attention launch");
   g_last_kernel = "generic_simt";
+  return SDPA_OK;
+}
+
+sdpa_status sdpa_forward_lse(const sdpa_params* p, const void* q, const void* k, const void* v, void* out,
+                             float* lse, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  sdpa::Problem P;
+  sdpa_status st = resolve(p, &P);
+  if (st != SDPA_OK) return st;
+  st = check_workspace(ws, ws_bytes, sdpa_workspace_size(p));
+  if (st != SDPA_OK) return st;
+  if ((long long)P.B * P.Lq * P.H == 0) return SDPA_OK;
+  if (!q || !out || !lse || (P.Lk > 0 && (!k || !v)))
+    return fail(SDPA_ERR_INVALID_ARG, "q, k, v, out and lse must not be NULL");
+  if ((p->flags & SDPA_FLAG_GENERIC_KERNEL) || P.bias || P.mask || P.bcls || !sdpa::prefill_supported(P, q, k, v, out))
+    return fail(SDPA_ERR_UNSUPPORTED,
+                "the row log-sum-exp comes from the tcgen05 kernel: bf16/fp16, qk_head_dim = v_head_dim = 64 or 128, "
+                "no bias, mask or block_info");
+  P.status = static_cast<int*>(ws);
+  P.lse = lse;
+  P.lse_out_mul = 0.69314718055994531f;  // natural log
+  const char* msg = nullptr;
+  cudaError_t e = sdpa::launch_prefill(P, q, k, v, out, nullptr, (cudaStream_t)stream, &msg);
+  if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");
+  g_last_kernel = "prefill_tcgen05";
   return SDPA_OK;
 }
 
@@ -410,6 +436,23 @@ size_t sdpa_backward_workspace_size(const sdpa_params* p) {
 sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, const void* v,
                           const void* out, const void* dout, void* dq, void* dk, void* dv,
                           float* dscale, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  return sdpa::backward(p, q, k, v, out, dout, nullptr, dq, dk, dv, dscale, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+sdpa_status sdpa_backward_lse(const sdpa_params* p, const void* q, const void* k, const void* v,
+                              const void* out, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              float* dscale, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  if (!lse) return fail(SDPA_ERR_INVALID_ARG, "lse must not be NULL");
+  return sdpa::backward(p, q, k, v, out, dout, lse, dq, dk, dv, dscale, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+}  // extern "C"
+
+namespace sdpa {
+
+sdpa_status backward(const sdpa_params* p, const void* q, const void* k, const void* v, const void* out,
+                     const void* dout, const float* lse_in, void* dq, void* dk, void* dv, float* dscale, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
   sdpa::Problem P;
   sdpa_status st = resolve(p, &P);
   if (st != SDPA_OK) return st;
@@ -427,15 +470,21 @@ sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, co
   void* scratch = static_cast<char*>(ws) + kStatusBytes;
   if (!(p->flags & SDPA_FLAG_GENERIC_KERNEL) && sdpa::backward_sm100_supported(P, q, k, v, out, dout, dq, dk, dv) &&
       sdpa::prefill_supported(P, q, k, v, dq)) {
-    // tcgen05: the forward again, for the row log-sum-exp (its output goes to dq, which the
-    // gradient overwrites), then delta, dK / dV and dQ / dscale
+    // tcgen05: the row log-sum-exp (the caller's, from sdpa_forward_lse, or the forward again,
+    // whose output goes to dq, which the gradient overwrites), then delta, dK / dV and dQ / dscale
     float* lse = static_cast<float*>(scratch);
     float* delta = lse + (size_t)P.B * P.H * P.Lq;
-    sdpa::Problem F = P;
-    F.lse = lse;
-    const char* msg = nullptr;
-    cudaError_t e = sdpa::launch_prefill(F, q, k, v, dq, nullptr, (cudaStream_t)stream, &msg);
-    if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");
+    cudaError_t e = cudaSuccess;
+    if (lse_in) {
+      lse = const_cast<float*>(lse_in);
+      P.lse_in_mul = 1.4426950408889634f;  // natural log -> log2 units
+    } else {
+      sdpa::Problem F = P;
+      F.lse = lse;
+      const char* msg = nullptr;
+      e = sdpa::launch_prefill(F, q, k, v, dq, nullptr, (cudaStream_t)stream, &msg);
+      if (e != cudaSuccess) return cuda_fail(e, msg ? msg : "prefill launch");
+    }
     e = sdpa::launch_backward_sm100(P, q, k, v, out, dout, dq, dk, dv, dscale, lse, delta, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "gradient launch");
     g_last_kernel = "backward_tcgen05";
@@ -452,6 +501,10 @@ sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, co
   g_last_kernel = "backward_simt";
   return SDPA_OK;
 }
+
+}  // namespace sdpa
+
+extern "C" {
 
 sdpa_status cache_update_at_index(void* k_cache, void* v_cache, const void* k_new,
                                   const void* v_new, sdpa_dtype dtype, int32_t d,

@@ -156,6 +156,16 @@ SDPA_API sdpa_status sdpa_workspace_init(void* ws, size_t ws_bytes, struct CUstr
 SDPA_API sdpa_status sdpa_forward(const sdpa_params* p, const void* q, const void* k, const void* v,
                          void* out, void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* sdpa_forward that also writes each query row's log-sum-exp, for a gradient that follows
+ * (sdpa_backward_lse) without running the forward again. lse: device float
+ * [batch][nheads][q_len], natural log, lse_i = log sum_j exp(logit_ij) over the keys row i
+ * attends; +inf for a row with no key or past q_lengths. Runs the tcgen05 kernel only:
+ * bf16/fp16, qk_head_dim = v_head_dim = 64 or 128, no bias, mask or block_info, no
+ * SDPA_FLAG_GENERIC_KERNEL (SDPA_ERR_UNSUPPORTED otherwise). Workspace as sdpa_forward. */
+SDPA_API sdpa_status sdpa_forward_lse(const sdpa_params* p, const void* q, const void* k, const void* v,
+                                      void* out, float* lse, void* ws, size_t ws_bytes,
+                                      struct CUstream_st* stream);
+
 /* Packed sequences (keywords q_segments, kv_segments and maxlen, paragraph "Packed
  * sequences"): nseg sequences stored one after the other along the sequence axis, with no
  * batch axis and no padding.
@@ -284,13 +294,27 @@ SDPA_API size_t sdpa_backward_workspace_size(const sdpa_params* p);
  *  - Arguments. mask, block_info, is_causal, q_offset, q_lengths and kv_lengths are as in
  *    sdpa_forward. A bias is SDPA_ERR_INVALID_ARG: the page's automatic differentiation
  *    takes the materialized implementation for a call with a bias. Head sizes are up to 256.
- *  - Kernels. bf16/fp16 with dqk = dv = 64 or 128 run two mma.sync tile kernels: dq (with the
- *    row log-sum-exp, delta = dout . out and dscale), then dk and dv per key tile. dscale is
- *    zeroed first with cudaMemsetAsync. Other types and sizes, or SDPA_FLAG_GENERIC_KERNEL,
- *    take three SIMT kernels, fp32 throughout. */
+ *  - Kernels. bf16/fp16 with dqk = dv = 128 and no mask or block_info run on tcgen05: the
+ *    forward kernel again for the row log-sum-exp (its output goes to dq, then overwritten),
+ *    delta = dout . out, then dk and dv per 128-key tile (resident in TMEM across the query
+ *    tiles of the group) and dq and dscale per 128-query tile. dx enters dk and dq as a 16-bit
+ *    high part plus the rounded remainder (two MMAs); w enters dv with one rounding. Other
+ *    bf16/fp16 calls with dqk = dv = 64 or 128 run two mma.sync tile kernels (dq with the row
+ *    log-sum-exp, delta and dscale, then dk and dv per key tile). Other types and sizes, or
+ *    SDPA_FLAG_GENERIC_KERNEL, take three SIMT kernels, fp32 throughout. dscale is zeroed
+ *    first with cudaMemsetAsync. */
 SDPA_API sdpa_status sdpa_backward(const sdpa_params* p, const void* q, const void* k, const void* v,
                                    const void* out, const void* dout, void* dq, void* dk, void* dv,
                                    float* dscale, void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* sdpa_backward given the row log-sum-exp that sdpa_forward_lse wrote for the same call (lse:
+ * device float [batch][nheads][q_len], natural log): the tcgen05 gradient then skips its own
+ * forward pass. Calls the tcgen05 gradient does not take ignore lse and run as sdpa_backward.
+ * Workspace as sdpa_backward. */
+SDPA_API sdpa_status sdpa_backward_lse(const sdpa_params* p, const void* q, const void* k, const void* v,
+                                       const void* out, const void* dout, const float* lse, void* dq, void* dk,
+                                       void* dv, float* dscale, void* ws, size_t ws_bytes,
+                                       struct CUstream_st* stream);
 
 /* Decoding with a KV cache (the page's example "decoding with a KV cache"; the Keras issue
  * "MultiHeadAttention is missing a position_bias call argument", cache_update_index):
@@ -380,10 +404,11 @@ SDPA_API sdpa_status sdpa_read_device_status(void* ws, struct CUstream_st* strea
 /* Message for the last non-OK status returned on this host thread. */
 SDPA_API const char* sdpa_last_error(void);
 
-/* Name of the kernel the last sdpa_forward / sdpa_forward_packed / sdpa_forward_with_weights /
- * sdpa_decode_with_cache / sdpa_backward call on this host thread launched for its attention
- * ("generic_simt", "prefill_tcgen05", "decode_splitkv", "weights_mma", "weights_simt",
- * "backward_mma", "backward_simt"). */
+/* Name of the kernel the last sdpa_forward / sdpa_forward_packed / sdpa_forward_lse /
+ * sdpa_forward_rope / sdpa_forward_with_weights / sdpa_decode_with_cache / sdpa_backward call on
+ * this host thread launched for its attention ("generic_simt", "prefill_tcgen05",
+ * "prefill_tcgen05_rope", "decode_splitkv", "weights_tcgen05", "weights_mma", "weights_simt",
+ * "backward_tcgen05", "backward_mma", "backward_simt"). */
 SDPA_API const char* sdpa_last_kernel(void);
 
 /* 1 in the range-checked build of the library (compiled with SDPA_DEBUG_CHECKS, shipped as

@@ -66,6 +66,8 @@ def load(path: str | None = None):
         lib = ctypes.CDLL(lib_path)
         lib.oracle_sdpa_forward.argtypes = [ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p]
         lib.oracle_sdpa_forward.restype = ctypes.c_int
+        lib.oracle_sdpa_forward_lse.argtypes = [ctypes.POINTER(_Problem), _f64p, _f64p, _f64p, _f64p, _f64p]
+        lib.oracle_sdpa_forward_lse.restype = ctypes.c_int
         lib.oracle_rope.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _i64p,
                                     ctypes.c_double, _f64p]
         lib.oracle_rope.restype = ctypes.c_int
@@ -138,9 +140,17 @@ def _broadcast4(a, dtype, batch, nheads, q_len, kv_len):
     return base, (sj, si, sh, sb)
 
 
+def sdpa_forward_lse(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_offset=0,
+                     q_lengths=None, kv_lengths=None, kv_head_rule: str = "contiguous", lib=None):
+    """sdpa_forward, and each row's log-sum-exp (natural log of the softmax's normaliser over the
+    attended keys; +inf for a row with no key or past q_lengths) as (B, H, Lq)."""
+    return sdpa_forward(q, k, v, bias, mask, scale, is_causal, q_offset, q_lengths, kv_lengths, kv_head_rule,
+                        lib, _with_lse=True)
+
+
 def sdpa_forward(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_offset=0,
                  q_lengths=None, kv_lengths=None, kv_head_rule: str = "contiguous",
-                 lib=None) -> np.ndarray:
+                 lib=None, _with_lse=False) -> np.ndarray:
     """scaled_dot_product_attention(query, key, value, [bias]; mask, scale, is_causal,
     q_offset, q_lengths, kv_lengths) in float64.
 
@@ -184,6 +194,13 @@ def sdpa_forward(q, k, v, bias=None, mask=None, scale=None, is_causal=False, q_o
         p.mask = _ptr(base, _u8p)
         p.mask_stride = (ctypes.c_int64 * 4)(*st)
     out = np.empty((B, Lq, H, Dv), dtype=np.float64)
+    if _with_lse:
+        lse = np.empty((B, H, Lq), dtype=np.float64)
+        rc = lib.oracle_sdpa_forward_lse(ctypes.byref(p), _ptr(q, _f64p), _ptr(k, _f64p),
+                                         _ptr(v, _f64p), _ptr(out, _f64p), _ptr(lse, _f64p))
+        if rc != 0:
+            raise OracleError(f"oracle_sdpa_forward_lse failed with code {rc}")
+        return out, lse
     rc = lib.oracle_sdpa_forward(ctypes.byref(p), _ptr(q, _f64p), _ptr(k, _f64p),
                                  _ptr(v, _f64p), _ptr(out, _f64p))
     if rc != 0:

@@ -76,10 +76,12 @@ static int check_problem(const oracle_sdpa_problem* p) {
   return ORACLE_OK;
 }
 
-/* One output row: batch b, query head h, query position i. `s` is scratch of kv_len doubles. */
+/* One output row: batch b, query head h, query position i. `s` is scratch of kv_len doubles.
+ * With `lse` not NULL it also receives the row's log-sum-exp, log sum_j exp(logit_j) over the
+ * attended keys (the softmax's normaliser), +inf for a row with no key or past q_lengths. */
 static void sdpa_row(const oracle_sdpa_problem* p, const double* q, const double* k,
                      const double* v, double* out, int64_t b, int64_t h, int64_t i,
-                     double* s, unsigned char* allowed) {
+                     double* s, unsigned char* allowed, double* lse) {
   const int64_t Lq = p->q_len, Lk = p->kv_len, H = p->nheads, Hkv = p->nkvheads;
   const int64_t D = p->dqk, Dv = p->dv;
   double* o = out + ((b * Lq + i) * H + h) * Dv;
@@ -88,6 +90,7 @@ static void sdpa_row(const oracle_sdpa_problem* p, const double* q, const double
   const int64_t qlen_b = p->q_lengths ? p->q_lengths[b] : Lq;
   if (i >= qlen_b) {
     for (int64_t e = 0; e < Dv; ++e) o[e] = 0.0;
+    if (lse) *lse = INFINITY;
     return;
   }
   /* Argument `kv_lengths`: the keys past kv_lengths[b] are not attended to. */
@@ -135,6 +138,7 @@ static void sdpa_row(const oracle_sdpa_problem* p, const double* q, const double
   /* A query attending to no key has a NaN output (fused-implementation paragraph). */
   if (n_allowed == 0) {
     for (int64_t e = 0; e < Dv; ++e) o[e] = NAN;
+    if (lse) *lse = INFINITY;
     return;
   }
 
@@ -145,6 +149,7 @@ static void sdpa_row(const oracle_sdpa_problem* p, const double* q, const double
     s[j] = exp(s[j] - m);
     denom += s[j];
   }
+  if (lse) *lse = m + log(denom);
   for (int64_t e = 0; e < Dv; ++e) o[e] = 0.0;
   for (int64_t j = 0; j < Lk; ++j) {
     if (!allowed[j]) continue;
@@ -155,9 +160,10 @@ static void sdpa_row(const oracle_sdpa_problem* p, const double* q, const double
 }
 
 /* scaled_dot_product_attention(query, key, value, [bias]; mask, scale, is_causal, q_offset,
- * q_lengths, kv_lengths): every (b, h, i) row of the output. */
-int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const double* k,
-                        const double* v, double* out) {
+ * q_lengths, kv_lengths): every (b, h, i) row of the output, and with `lse` not NULL each row's
+ * log-sum-exp, [batch][nheads][q_len]. */
+int oracle_sdpa_forward_lse(const oracle_sdpa_problem* p, const double* q, const double* k,
+                            const double* v, double* out, double* lse) {
   int rc = check_problem(p);
   if (rc) return rc;
   if (p->batch == 0 || p->q_len == 0) return ORACLE_OK;
@@ -176,13 +182,18 @@ int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const dou
         const int64_t b = r / (p->nheads * p->q_len);
         const int64_t h = (r / p->q_len) % p->nheads;
         const int64_t i = r % p->q_len;
-        sdpa_row(p, q, k, v, out, b, h, i, s, allowed);
+        sdpa_row(p, q, k, v, out, b, h, i, s, allowed, lse ? lse + (b * p->nheads + h) * p->q_len + i : NULL);
       }
     }
     free(s);
     free(allowed);
   }
   return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+int oracle_sdpa_forward(const oracle_sdpa_problem* p, const double* q, const double* k,
+                        const double* v, double* out) {
+  return oracle_sdpa_forward_lse(p, q, k, v, out, NULL);
 }
 
 /* Rotary position embedding of query or key rows (the Keras thread "MultiHeadAttention is

@@ -434,6 +434,39 @@ def rope_pairs_halves_with_geometric_frequencies(lib):
     _close(angles[1:] / angles[:-1], np.full(d // 2 - 1, base ** (-2 / d)), 1e-12)
 
 
+# ---- the row log-sum-exp (the softmax's normaliser) ----------------------------------------
+
+@pin
+def lse_is_torch_logsumexp_of_the_masked_logits(lib):
+    """oracle.sdpa_forward_lse's lse is PyTorch's float64 logsumexp over each row's attended
+    logits (scale q.k + bias, causal with offsets, lengths, GQA through repeated heads), +inf for
+    a row with no key and for padding rows; the output equals the plain forward's; and the
+    weights exp(logit - lse) of a row add up to 1."""
+    rng = _rng(91)
+    B, Lq, Lk, H, Hkv, D = 2, 9, 12, 4, 2, 8
+    q, k, v = _qkv(rng, B, Lq, Lk, H, Hkv, D)
+    bias = rng.standard_normal((1, H, Lq, Lk))
+    kw = dict(bias=bias, is_causal=True, q_offset=[2, -3], q_lengths=[9, 6], kv_lengths=[12, 10], scale=0.4)
+    out, lse = oracle.sdpa_forward_lse(q, k, v, lib=lib, **kw)
+    _close(out, oracle.sdpa_forward(q, k, v, lib=lib, **kw), 0.0)
+    kr = np.repeat(k, H // Hkv, axis=2)
+    logits = 0.4 * np.einsum("bihd,bjhd->bhij", q, kr) + bias
+    i = np.arange(Lq)[:, None]
+    j = np.arange(Lk)[None, :]
+    for b, (off, ql, kl) in enumerate(zip([2, -3], [9, 6], [12, 10])):
+        allowed = (j <= off + i) & (j < kl) & (i < ql)
+        x = torch.from_numpy(np.where(allowed[None], logits[b], -np.inf))
+        want = torch.logsumexp(x, dim=-1).numpy()
+        want = np.where(np.isneginf(want), np.inf, want)  # no key: +inf
+        want[:, ql:] = np.inf  # padding rows: +inf
+        assert np.array_equal(np.isinf(lse[b]), np.isinf(want))
+        fin = np.isfinite(want)
+        _close(lse[b][fin], want[fin], 1e-12)
+        w = np.where(allowed[None], np.exp(logits[b] - lse[b][..., None]), 0.0)
+        rows = fin
+        _close(w.sum(-1)[rows], np.ones(int(rows.sum())), 1e-12)
+
+
 # ---- with weights and fdrop (the entry's "See also"; argument fdrop) -------------------------
 
 @pin

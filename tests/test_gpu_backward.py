@@ -155,3 +155,30 @@ def test_backward_full_size_sampled():
         assert_close_rel(dq[b:b + 1, :, hs], wq, 1e-2, f"dq b={b} kv head {kvh}")
         assert_close_rel(dk[b:b + 1, :, kvh:kvh + 1], wk, 1e-2, f"dk b={b} kv head {kvh}")
         assert_close_rel(dv[b:b + 1, :, kvh:kvh + 1], wv, 1e-2, f"dv b={b} kv head {kvh}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_forward_lse_and_backward_from_it(dtype):
+    """sdpa_forward_lse's row log-sum-exp against the oracle's (natural log, +inf for rows with
+    no key or past q_lengths), and the gradient that takes it instead of running the forward
+    again, against the oracle's gradient."""
+    q, k, v, dout = _inputs(17, 3, 200, 270, 4, 2, 128, 128, dtype)
+    kw = dict(is_causal=True, q_offset=[20, -5, 0], q_lengths=[200, 131, 12], kv_lengths=[270, 140, 0])
+    qd, kd, vd, dd = (t.to(DEV) for t in (q, k, v, dout))
+    out, lse = sdpa.sdpa_forward_lse(qd, kd, vd, **kw)
+    assert sdpa.read_device_status() == sdpa.SDPA_OK
+    want_o, want_lse = oracle.sdpa_forward_lse(f64(q), f64(k), f64(v), **kw)
+    got = lse.cpu().double().numpy()
+    assert np.array_equal(np.isinf(got), np.isinf(want_lse)), "lse: +inf pattern differs"
+    fin = np.isfinite(want_lse)
+    assert np.abs(got[fin] - want_lse[fin]).max() <= 1e-4
+    fwd = sdpa.sdpa_forward(qd, kd, vd, **kw)
+    assert torch.equal(torch.nan_to_num(out), torch.nan_to_num(fwd))  # the same output
+    dq, dk, dv, ds = sdpa.sdpa_backward(qd, kd, vd, out, dd, lse=lse, **kw)
+    assert sdpa.last_kernel() == "backward_tcgen05"
+    assert sdpa.read_device_status() == sdpa.SDPA_OK
+    wq, wk, wv, wds = oracle.sdpa_backward(f64(q), f64(k), f64(v), f64(dout), **kw)
+    for name, g, w in (("dq", dq, wq), ("dk", dk, wk), ("dv", dv, wv)):
+        assert_close_rel(g, w, 1e-2, f"lse path {name}")
+    mag = float(np.abs((f64(q) * wq).sum(axis=-1)).sum()) * np.sqrt(q.shape[-1])
+    assert abs(float(ds) - wds) <= 1e-2 * max(1.0, mag)

@@ -38,6 +38,7 @@ MUTANTS = {
     "rope_sin_sign": ("o[c] = x0 * cos(a) - x1 * sin(a);", "o[c] = x0 * cos(a) + x1 * sin(a);"),
     "rope_frequency_exponent": ("pow(base, -2.0 * (double)c / (double)d)", "pow(base, -1.0 * (double)c / (double)d)"),
     "weights_dropout_unscaled": ("? w / (1.0 - drop_p) : 0.0", "? w : 0.0"),
+    "lse_without_max": ("  if (lse) *lse = m + log(denom);", "  if (lse) *lse = log(denom);"),
     "weights_dropout_inverted": ("dropout_keep(seed, base + (uint64_t)j, thr) ?", "!dropout_keep(seed, base + (uint64_t)j, thr) ?"),
     "weights_dropout_same_draw_per_group": ("fmix64(index >> 2));\n  const uint32_t u = (uint32_t)(r >> (16 * (index & 3)))",
                                             "fmix64(index >> 2));\n  const uint32_t u = (uint32_t)(r >> 0)"),
