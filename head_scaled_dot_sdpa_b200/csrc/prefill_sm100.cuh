@@ -49,6 +49,12 @@ using namespace sm100;
 
 constexpr int kBlockM = 128;
 constexpr int kBlockN = 128;
+// With head_dim 64, P is handed to the MMA warp in two parts: the first kEarlyKeys keys as
+// soon as they are written (their PV steps start while the softmax finishes the rest), then the
+// remainder. (With head_dim 128 the split was measured 1-2% slower and P goes in one part.)
+constexpr int kEarlyKeys = 96;
+template <int D>
+constexpr bool kSplitP = D == 64;
 constexpr int kThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer + MMA (+2 idle)
 // Register split (setmaxnreg): the two softmax warpgroups grow to kSoftmaxRegs, the last one
 // shrinks to kOtherRegs. 2*128*216 + 128*72 = 64512 = 384 * 168, the launch's registers; the
@@ -95,7 +101,7 @@ struct Cfg {
   static constexpr int kQSlots = 2;
   static constexpr int kBiasBytes = kBT ? 2 * kBiasSlots * kBiasTileBytes : 0;
   static constexpr int kBarriers =
-      3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots;
+      3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots + 2;
   // tiles (+ the bias tiles), barriers, unit ring, TMEM address, abort flag, and slack to align
   // the base to 1024 bytes
   static constexpr int smem_bytes() {
@@ -316,7 +322,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint64_t* q_rot = drain + 1;                   // [kQSlots] Q tile rotated (P.q_rope)
   uint64_t* unit_full = q_rot + C::kQSlots;      // [kUnitSlots]
   uint64_t* unit_empty = unit_full + kUnitSlots; // [kUnitSlots]
-  int* unit_ring = reinterpret_cast<int*>(unit_empty + kUnitSlots);
+  uint64_t* p_early = unit_empty + kUnitSlots;  // [2] the first kEarlyKeys keys of P written
+  int* unit_ring = reinterpret_cast<int*>(p_early + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring + kUnitSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // MMA groups issued so far by the MMA warp of tile A / tile B (the turn order below)
@@ -334,6 +341,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4);  // one arrive per softmax warp
+      mbar_init(&p_early[s], 4);
       mbar_init(&o_ready[s], 1);
       mbar_init(&o_free[s], 4);
     }
@@ -592,26 +600,52 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           const int vs = x % C::kVStages;
           if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
           if (first && !wait_all(&o_free[s], (oc & 1) ^ 1)) return false;
-          return wait_all(&p_full[s], (sc - 1) & 1);
+          return wait_all(kSplitP<D> ? &p_early[s] : &p_full[s], (sc - 1) & 1);
         };
-        // O += P(x) V(x) for this tile's key tile at ring position x (after pv_ready); `last`:
-        // the group ends here and is published
-        auto pv = [&](uint32_t x, bool first, bool last) {
+        // O += P(x) V(x) for this tile's key tile at ring position x (after pv_ready): the steps
+        // over the first kEarlyKeys keys, then, once the rest of P is written, the others (they
+        // queue behind the first ones on a tensor pipe that is still busy); `last`: the group
+        // ends here and is published
+        auto pv = [&](uint32_t x, bool first, bool last) -> bool {
           const int vs = x % C::kVStages;
-          tc_fence_after();
-          if (elected) {
-            const uint32_t vtile = v_base + vs * C::kTileBytes;
+          const uint32_t vtile = v_base + vs * C::kTileBytes;
+          // B = V (keys x dims, dims contiguous): MN-major; 64-dim regions kRegionBytes apart
+          // (LBO), 8-key groups 1024 bytes apart (SBO); 16 keys per step.
+          auto steps = [&](int k0, int k1) {
 #pragma unroll
-            for (int kk = 0; kk < kBlockN / 16; ++kk) {
-              // B = V (keys x dims, dims contiguous): MN-major; 64-dim regions kRegionBytes
-              // apart (LBO), 8-key groups 1024 bytes apart (SBO); 16 keys per step.
+            for (int kk = k0; kk < k1; ++kk) {
               const uint64_t bdesc = smem_desc_sw128(vtile + kk * 16 * 128, kRegionBytes, 1024);
               mma_ts(o_tmem, s_tmem + kk * 8, bdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
             }
-            if (last) publish();
-            mma_commit(&v_empty[vs]);
+          };
+          tc_fence_after();
+          if constexpr (!kSplitP<D>) {
+            if (elected) {
+              steps(0, kBlockN / 16);
+              if (last) publish();
+              mma_commit(&v_empty[vs]);
+            }
+            __syncwarp();
+            return true;
           }
-          __syncwarp();
+          uint32_t ok = 1;
+          if (elected) {
+            steps(0, kEarlyKeys / 16);
+            // the rest of P is usually written while the first steps run: the issuing lane
+            // alone waits for it, so that the remaining steps follow on a still busy pipe
+            ok = mbar_wait(&p_full[s], (sc - 1) & 1, tmo, abort_flag) ? 1u : 0u;
+            if (ok) {
+              tc_fence_after();
+              steps(kEarlyKeys / 16, kBlockN / 16);
+              if (last) publish();
+              mma_commit(&v_empty[vs]);
+            }
+          }
+          if (__shfl_sync(0xffffffffu, ok, 0) == 0) {
+            fail();
+            return false;
+          }
+          return true;
         };
         int ja = 0, jb = 0, jm = 0;
         uint32_t k_grp = 0;  // groups of this tile issued in this unit
@@ -631,7 +665,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if (pend) {
               if (!pv_ready(prev, first_pv)) return;
               if (!turn_wait(before(k_grp))) return;
-              pv(prev, first_pv, true);
+              if (!pv(prev, first_pv, true)) return;
               ++mine;
               ++k_grp;
               first_pv = false;
@@ -646,7 +680,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if (pend && !pv_ready(prev, first_pv)) return;
             if (!turn_wait(before(k_grp))) return;
             // PV of this tile's previous key tile first: S(x) overwrites the P it reads
-            if (pend) pv(prev, first_pv, false);
+            if (pend && !pv(prev, first_pv, false)) return;
             if (pend) first_pv = false;
             tc_fence_after();
             if (elected) {
@@ -679,7 +713,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if (pend) {
           if (!pv_ready(prev, first_pv)) return;
           if (!turn_wait(before(k_grp))) return;
-          pv(prev, first_pv, true);
+          if (!pv(prev, first_pv, true)) return;
           ++mine;
           ++k_grp;
         }
@@ -840,7 +874,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[s]);
+            if (lane == 0) {
+              if constexpr (kSplitP<D>) mbar_arrive(&p_early[s]);
+              mbar_arrive(&p_full[s]);
+            }
             continue;
           }
           // Fast path (no bias, no mask bytes, every key of the tile attended by every row of
@@ -1013,13 +1050,27 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             }
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[c / 2][(c % 2) * 16 + e] = pk[e];
+            if (kSplitP<D> && c == kEarlyKeys / 32 - 1) {
+              // keys [0, kEarlyKeys): 16-bit pairs in columns [0, kEarlyKeys / 2)
+              static_assert(kEarlyKeys == 96, "P columns stored early: 32 + 16");
+              tmem_st32(lane_addr + scol, v[0]);
+              tmem_st16(lane_addr + scol + 32, *reinterpret_cast<const uint32_t(*)[16]>(&v[1][0]));
+              tmem_wait_st();
+              tc_fence_before();
+              __syncwarp();  // the warp's stores are done (each lane waited for its own)
+              if (lane == 0) mbar_arrive(&p_early[s]);
+            }
           }
           l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-          tmem_st32(lane_addr + scol, v[0]);
-          tmem_st32(lane_addr + scol + 32, v[1]);
+          if constexpr (kSplitP<D>) {
+            tmem_st16(lane_addr + scol + kEarlyKeys / 2, *reinterpret_cast<const uint32_t(*)[16]>(&v[1][16]));
+          } else {
+            tmem_st32(lane_addr + scol, v[0]);
+            tmem_st32(lane_addr + scol + 32, v[1]);
+          }
           tmem_wait_st();
           tc_fence_before();
-          __syncwarp();  // the warp's stores are done (each lane waited for its own)
+          __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[s]);
         }
         if (!wait_all(&o_ready[s], oc & 1)) return;

@@ -6,7 +6,8 @@
 // An HBM-bound elementwise pass. The angle of (row t, pair c) is the same for every head, so one
 // thread takes VEC consecutive pairs of one row, computes their sines and cosines once and
 // rotates those pairs in all nheads heads; the threads of a warp cover consecutive pairs, so
-// each head's two halves are read and written in coalesced runs (VEC = 2: 4-byte 16-bit pairs).
+// each head's two halves are read and written in coalesced runs (VEC = 8: 16-byte runs of
+// 16-bit values, four heads' loads in flight at a time).
 // The frequencies base^(-2c/d) are a per-block table in double precision. The angle is formed
 // and reduced to [-pi, pi] in double precision (positions of 10^5 and more keep their accuracy),
 // then CUDA's sincosf evaluates it in single precision. Each element is read before it is
@@ -44,36 +45,48 @@ rope_kernel(const T* x, T* out, long long rows, int nheads, int d, const int32_t
     }
     const T* xr = x + t * row_elems + c0;
     T* orow = out + t * row_elems + c0;
-    for (int h = 0; h < nheads; ++h) {
-      float x0[VEC], x1[VEC];
-      if constexpr (VEC == 2 && sizeof(T) == 2) {
-        const uint32_t a = *reinterpret_cast<const uint32_t*>(xr + (long long)h * d);
-        const uint32_t b = *reinterpret_cast<const uint32_t*>(xr + (long long)h * d + half);
-        const T* pa = reinterpret_cast<const T*>(&a);
-        const T* pb = reinterpret_cast<const T*>(&b);
-        x0[0] = to_f32(pa[0]); x0[1] = to_f32(pa[1]);
-        x1[0] = to_f32(pb[0]); x1[1] = to_f32(pb[1]);
-      } else {
+    if constexpr (VEC == 8 && sizeof(T) == 2) {
+      // 16 bytes of each half per head; four heads' loads in flight before their stores
+      constexpr int kHeads = 4;
+      for (int h0 = 0; h0 < nheads; h0 += kHeads) {
+        uint4 a[kHeads], b[kHeads];
+#pragma unroll
+        for (int g = 0; g < kHeads; ++g) {
+          if (h0 + g < nheads) {
+            a[g] = *reinterpret_cast<const uint4*>(xr + (long long)(h0 + g) * d);
+            b[g] = *reinterpret_cast<const uint4*>(xr + (long long)(h0 + g) * d + half);
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < kHeads; ++g) {
+          if (h0 + g >= nheads) break;
+          const T* pa = reinterpret_cast<const T*>(&a[g]);
+          const T* pb = reinterpret_cast<const T*>(&b[g]);
+          uint4 ya, yb;
+          T* qa = reinterpret_cast<T*>(&ya);
+          T* qb = reinterpret_cast<T*>(&yb);
+#pragma unroll
+          for (int u = 0; u < VEC; ++u) {
+            const float x0 = to_f32(pa[u]), x1 = to_f32(pb[u]);
+            qa[u] = from_f32<T>(x0 * cs[u] - x1 * sn[u]);
+            qb[u] = from_f32<T>(x1 * cs[u] + x0 * sn[u]);
+          }
+          *reinterpret_cast<uint4*>(orow + (long long)(h0 + g) * d) = ya;
+          *reinterpret_cast<uint4*>(orow + (long long)(h0 + g) * d + half) = yb;
+        }
+      }
+    } else {
+      for (int h = 0; h < nheads; ++h) {
+        float x0[VEC], x1[VEC];
 #pragma unroll
         for (int u = 0; u < VEC; ++u) {
           x0[u] = to_f32(xr[(long long)h * d + u]);
           x1[u] = to_f32(xr[(long long)h * d + half + u]);
         }
-      }
-      T y0[VEC], y1[VEC];
-#pragma unroll
-      for (int u = 0; u < VEC; ++u) {
-        y0[u] = from_f32<T>(x0[u] * cs[u] - x1[u] * sn[u]);
-        y1[u] = from_f32<T>(x1[u] * cs[u] + x0[u] * sn[u]);
-      }
-      if constexpr (VEC == 2 && sizeof(T) == 2) {
-        *reinterpret_cast<uint32_t*>(orow + (long long)h * d) = *reinterpret_cast<const uint32_t*>(y0);
-        *reinterpret_cast<uint32_t*>(orow + (long long)h * d + half) = *reinterpret_cast<const uint32_t*>(y1);
-      } else {
 #pragma unroll
         for (int u = 0; u < VEC; ++u) {
-          orow[(long long)h * d + u] = y0[u];
-          orow[(long long)h * d + half + u] = y1[u];
+          orow[(long long)h * d + u] = from_f32<T>(x0[u] * cs[u] - x1[u] * sn[u]);
+          orow[(long long)h * d + half + u] = from_f32<T>(x1[u] * cs[u] + x0[u] * sn[u]);
         }
       }
     }
@@ -88,16 +101,16 @@ cudaError_t launch_t(const void* x, void* out, long long rows, int nheads, int d
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // 16-bit pairs of two consecutive c: both halves of every row start on a 4-byte boundary when
-  // half is even and the arrays are 4-byte aligned
-  const bool vec2 = sizeof(T) == 2 && half % 2 == 0 && (reinterpret_cast<uintptr_t>(x) % 4 == 0) &&
-                    (reinterpret_cast<uintptr_t>(out) % 4 == 0);
-  const long long items = rows * (vec2 ? half / 2 : half);
+  // 16-bit rows whose halves are whole 16-byte runs (half a multiple of 8, 16-byte aligned
+  // arrays): 8 consecutive pairs per thread; otherwise one pair per thread
+  const bool vec8 = sizeof(T) == 2 && half % 8 == 0 && (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
+                    (reinterpret_cast<uintptr_t>(out) % 16 == 0);
+  const long long items = rows * (vec8 ? half / 8 : half);
   const long long blocks = (items + kThreads - 1) / kThreads;
   const unsigned grid = (unsigned)(blocks < 8LL * sms ? blocks : 8LL * sms);
   const size_t smem = sizeof(double) * half;
-  if (vec2)
-    rope_kernel<T, 2><<<grid, kThreads, smem, stream>>>((const T*)x, (T*)out, rows, nheads, d, positions, log2(base));
+  if (vec8)
+    rope_kernel<T, 8><<<grid, kThreads, smem, stream>>>((const T*)x, (T*)out, rows, nheads, d, positions, log2(base));
   else
     rope_kernel<T, 1><<<grid, kThreads, smem, stream>>>((const T*)x, (T*)out, rows, nheads, d, positions, log2(base));
   return cudaGetLastError();
