@@ -40,21 +40,25 @@ __device__ __forceinline__ bool checked(int* status, bool ok) {
 #define SDPA_CHECKED(status, cond) (true)
 #endif
 
-// The dropout draw of scaled_dot_product_attention_with_weights (argument fdrop as dropout).
-// The weights' row-major positions (b, h, i, j) are taken four at a time: the group
-// index / 4 gets r = fmix64(seed + fmix64(index / 4)), fmix64 being the 64-bit finalizer of
-// Austin Appleby's MurmurHash3, and the weight at `index` takes 16-bit field index % 4 of r
-// (lowest first) as u in [0, 2^16); it is kept when u >= ceil(p * 2^16).
-__device__ __forceinline__ unsigned long long fmix64(unsigned long long k) {
-  k ^= k >> 33;
-  k *= 0xff51afd7ed558ccdULL;
-  k ^= k >> 33;
-  k *= 0xc4ceb9fe1a85ec53ULL;
-  k ^= k >> 33;
-  return k;
+// The dropout draw of scaled_dot_product_attention_with_weights (argument fdrop as dropout):
+// SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) used as a counter-based generator. Its n-th
+// output from state `seed` is splitmix64_mix(seed + n * kSplitMixGamma). The weights' row-major
+// positions (b, h, i, j) are taken four at a time: group g = index / 4 gets output n = g + 1,
+// and the weight at `index` takes 16-bit field index % 4 of it (lowest first) as u in
+// [0, 2^16); it is kept when u >= ceil(p * 2^16). Consecutive groups differ by one gamma in
+// the mixed state, so a run of groups costs one 64-bit add and one mix each.
+constexpr unsigned long long kSplitMixGamma = 0x9e3779b97f4a7c15ULL;
+__device__ __forceinline__ unsigned long long splitmix64_mix(unsigned long long z) {
+  z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ULL;
+  z = (z ^ (z >> 27)) * 0x94d049bb133111ebULL;
+  return z ^ (z >> 31);
+}
+// the state that gives group g's draw
+__device__ __forceinline__ unsigned long long dropout_state(unsigned long long seed, unsigned long long group) {
+  return seed + (group + 1) * kSplitMixGamma;
 }
 __device__ __forceinline__ unsigned long long dropout_group_draw(unsigned long long seed, unsigned long long group) {
-  return fmix64(seed + fmix64(group));
+  return splitmix64_mix(dropout_state(seed, group));
 }
 // bits f of the result: whether field f (f < 4) of r is kept
 __device__ __forceinline__ uint32_t dropout_keep4(unsigned long long r, unsigned threshold) {

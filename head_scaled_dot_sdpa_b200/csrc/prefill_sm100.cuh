@@ -841,9 +841,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               uint32_t keep = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
               if (P.drop_thr > 0) {
                 uint32_t kd = 0;
-                const unsigned long long g0 = (wbase + (unsigned long long)(key0 + 32 * c)) >> 2;
+                // the 8 groups of these 32 keys: consecutive draws, one gamma apart
+                unsigned long long z = dropout_state(P.drop_seed, (wbase + (unsigned long long)(key0 + 32 * c)) >> 2);
 #pragma unroll
-                for (int gq = 0; gq < 8; ++gq) kd |= dropout_keep4(dropout_group_draw(P.drop_seed, g0 + gq), P.drop_thr) << (4 * gq);
+                for (int gq = 0; gq < 8; ++gq, z += kSplitMixGamma)
+                  kd |= dropout_keep4(splitmix64_mix(z), P.drop_thr) << (4 * gq);
                 keep &= kd;
               }
               const float sc_keep = P.drop_thr > 0 ? P.inv_keep : 1.f;

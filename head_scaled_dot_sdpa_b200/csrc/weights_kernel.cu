@@ -8,11 +8,11 @@
 // [batch][nheads][q_len][kv_len], in the input type. A row with no attended key has NaN weights
 // and output; a row past q_lengths has zero weights and output.
 //
-// The dropout draw is counter-based: the weights' row-major positions are taken four at a
-// time, the group index / 4 gets r = fmix64(seed + fmix64(index / 4)) (fmix64: the 64-bit
-// finalizer of Austin Appleby's MurmurHash3), and the weight at `index` takes the 16-bit field
-// number index % 4 of r (lowest first) as u in [0, 2^16); it is kept when
-// u >= ceil(p * 2^16), an integer comparison.
+// The dropout draw is counter-based (SplitMix64, device_common.cuh): the weights' row-major
+// positions are taken four at a time, group g = index / 4 gets the generator's output g + 1
+// from state seed, and the weight at `index` takes the 16-bit field number index % 4 of it
+// (lowest first) as u in [0, 2^16); it is kept when u >= ceil(p * 2^16), an integer
+// comparison.
 //
 // Two kernels:
 //  - weights_mma_kernel (bf16/fp16, head_dim = v_head_dim = 64 or 128): one CTA per

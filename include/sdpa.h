@@ -219,8 +219,9 @@ SDPA_API sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed
  *    key has NaN weights and output. A row past q_lengths has zero weights and output.
  *  - The dropout keeps w_ij, divided by 1 - drop_p, when its draw u >= ceil(drop_p * 2^16),
  *    and otherwise sets it to 0. The weights' row-major positions are taken four at a time:
- *    the group index / 4 gets r = fmix64(seed + fmix64(index / 4)), fmix64 being the 64-bit
- *    finalizer of MurmurHash3, and u is the 16-bit field index % 4 of r (lowest first). So a
+ *    group g = index / 4 gets r = mix(seed + (g + 1) * 0x9e3779b97f4a7c15), the SplitMix64
+ *    generator's output g + 1 from state seed (mix: its finalizer, Steele, Lea and Flood 2014),
+ *    and u is the 16-bit field index % 4 of r (lowest first). So a
  *    weight is kept with probability 1 - ceil(drop_p * 2^16) / 2^16, within 2^-16 of
  *    1 - drop_p. drop_p must be in [0, 1), and 0 means no dropout.
  *  - out = weights · v.

@@ -223,22 +223,20 @@ int oracle_rope(const double* x, int64_t rows, int64_t nheads, int64_t d, const 
   return ORACLE_OK;
 }
 
-/* Counter-based dropout draw. The weights' linear indices (b, h, i, j), row-major, are taken
- * four at a time: the group index / 4 gets one 64-bit value from the 64-bit finalizer of Austin
- * Appleby's MurmurHash3 ("fmix64"), applied to the group and then to that plus the seed, and
- * the weight at `index` takes its 16-bit field number index % 4 (lowest first) as an integer u
- * in [0, 2^16). The weight is kept when u >= threshold = ceil(drop_p * 2^16): with probability
- * 1 - threshold / 2^16, within 2^-16 of 1 - drop_p. */
-static uint64_t fmix64(uint64_t k) {
-  k ^= k >> 33;
-  k *= 0xff51afd7ed558ccdULL;
-  k ^= k >> 33;
-  k *= 0xc4ceb9fe1a85ec53ULL;
-  k ^= k >> 33;
-  return k;
+/* Counter-based dropout draw: SplitMix64 (Steele, Lea and Flood, "Fast splittable pseudorandom
+ * number generators", OOPSLA 2014). Its n-th output (n = 1, 2, ...) from state `seed` is the
+ * mixing function applied to seed + n * gamma, gamma = 0x9e3779b97f4a7c15. The weights' linear
+ * indices (b, h, i, j), row-major, are taken four at a time: group g = index / 4 gets output
+ * n = g + 1, and the weight at `index` takes its 16-bit field number index % 4 (lowest first)
+ * as an integer u in [0, 2^16). The weight is kept when u >= threshold = ceil(drop_p * 2^16):
+ * with probability 1 - threshold / 2^16, within 2^-16 of 1 - drop_p. */
+static uint64_t splitmix64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ULL;
+  z = (z ^ (z >> 27)) * 0x94d049bb133111ebULL;
+  return z ^ (z >> 31);
 }
 static int dropout_keep(uint64_t seed, uint64_t index, uint32_t threshold) {
-  const uint64_t r = fmix64(seed + fmix64(index >> 2));
+  const uint64_t r = splitmix64_mix(seed + ((index >> 2) + 1) * 0x9e3779b97f4a7c15ULL);
   const uint32_t u = (uint32_t)(r >> (16 * (index & 3))) & 0xFFFFu;
   return u >= threshold;
 }

@@ -40,8 +40,8 @@ MUTANTS = {
     "weights_dropout_unscaled": ("? w / (1.0 - drop_p) : 0.0", "? w : 0.0"),
     "lse_without_max": ("  if (lse) *lse = m + log(denom);", "  if (lse) *lse = log(denom);"),
     "weights_dropout_inverted": ("dropout_keep(seed, base + (uint64_t)j, thr) ?", "!dropout_keep(seed, base + (uint64_t)j, thr) ?"),
-    "weights_dropout_same_draw_per_group": ("fmix64(index >> 2));\n  const uint32_t u = (uint32_t)(r >> (16 * (index & 3)))",
-                                            "fmix64(index >> 2));\n  const uint32_t u = (uint32_t)(r >> 0)"),
+    "weights_dropout_same_draw_per_group": ("0x9e3779b97f4a7c15ULL);\n  const uint32_t u = (uint32_t)(r >> (16 * (index & 3)))",
+                                            "0x9e3779b97f4a7c15ULL);\n  const uint32_t u = (uint32_t)(r >> 0)"),
     "weights_head_batch_swapped": ("double* wrow = weights + ((b * H + h) * Lq + i) * Lk;",
                                    "double* wrow = weights + ((h * B + b) * Lq + i) * Lk;"),
     "backward_delta_sign": ("x[j] * (dw[j] - wdw)", "x[j] * (dw[j] + wdw)"),
