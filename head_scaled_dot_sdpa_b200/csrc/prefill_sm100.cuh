@@ -69,6 +69,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 bytes (64 16-bit columns)
 constexpr int kNone = 1 << 30;
 constexpr int kUnitSlots = 4;        // ring of unit indices handed from the producer to the others
+constexpr int kUnitInfoBytes = 128;  // per ring slot: the unit's decomposition (struct Unit)
 constexpr int kUnitConsumers = 10;   // the two MMA warps and the 8 softmax warps
 constexpr int kMmaWarpA = 9, kMmaWarpB = 11;  // MMA issuers of tile A and tile B
 constexpr int kSchedWord = 16;       // int offset in the status area of the unit counter (+1: done)
@@ -105,7 +106,8 @@ struct Cfg {
   // tiles (+ the bias tiles), barriers, unit ring, TMEM address, abort flag, and slack to align
   // the base to 1024 bytes
   static constexpr int smem_bytes() {
-    return (kQSlots + kKStages + kVStages) * kTileBytes + kBiasBytes + kBarriers * 8 + 64 + 1024;
+    return (kQSlots + kKStages + kVStages) * kTileBytes + kBiasBytes + kBarriers * 8 + 64 +
+           kUnitSlots * kUnitInfoBytes + 16 + 1024;
   }
 };
 static_assert(Cfg<64, true>::smem_bytes() <= 227 * 1024, "bias tiles fit for head_dim 64");
@@ -131,6 +133,7 @@ struct Unit {
   long long o0;     // first row of the sequence in out viewed as (rows, heads, head_dim)
   QTile t[2];
 };
+static_assert(sizeof(Unit) <= kUnitInfoBytes, "unit ring slot");
 
 __device__ __forceinline__ QTile make_qtile(const Problem& P, const BatchInfo& bi, int h, int qt, bool present) {
   QTile x;
@@ -328,6 +331,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // MMA groups issued so far by the MMA warp of tile A / tile B (the turn order below)
   volatile uint32_t* issued = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);  // [2]
+  // the decomposition of the unit in each ring slot, written by the producer with the index
+  Unit* unit_info = reinterpret_cast<Unit*>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint64_t tmo = P.wait_timeout_ns;
@@ -395,10 +400,12 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   // Dynamic scheduling: the producer takes units from a counter in the workspace (units are
   // numbered longest causal rows first) and hands them to the other roles through a small ring.
   unsigned int* sched = reinterpret_cast<unsigned int*>(P.status) + kSchedWord;
-  auto next_unit = [&](uint32_t k, int& u) -> bool {  // consumers: the k-th unit of this CTA
+  // consumers: the k-th unit of this CTA and its decomposition (copied before the slot is released)
+  auto next_unit = [&](uint32_t k, int& u, Unit& w) -> bool {
     const int slot = k % kUnitSlots;
     if (!wait_all(&unit_full[slot], (k / kUnitSlots) & 1)) return false;
     u = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+    if (u < n_units) w = unit_info[slot];
     __syncwarp();
     if (elected) mbar_arrive(&unit_empty[slot]);
     return true;
@@ -425,14 +432,18 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if (!wait_all(&unit_empty[slot], ((k / kUnitSlots) & 1) ^ 1)) return;
         int u = 0;
         if (elected) {
+          // the unit's decomposition is computed once, here, and handed over with its index:
+          // its integer divisions stay off the MMA and softmax warps' path between units
           u = (int)atomicAdd(sched, 1u);
           if (u > n_units) u = n_units;
+          if (u < n_units) unit_info[slot] = make_unit(P, u);
           unit_ring[slot] = u;
           mbar_arrive(&unit_full[slot]);
         }
         u = __shfl_sync(0xffffffffu, u, 0);
         if (u >= n_units) break;
-        const Unit w = make_unit(P, u);
+        __syncwarp();
+        const Unit w = unit_info[slot];
         if (w.t[0].n == 0 && w.t[1].n == 0) continue;
         // The unit's Q tiles come from DRAM (each is read once); their slots free only when
         // the previous unit's last S completes, so they are first brought into L2 now, about
@@ -571,9 +582,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       uint32_t g = 0, sc = 0, qi = 0, oc = 0;  // qi: Q tiles of both streams so far (ring position)
       for (uint32_t kq = 0;; ++kq) {
         int u;
-        if (!next_unit(kq, u)) return;
+        Unit w;
+        if (!next_unit(kq, u, w)) return;
         if (u >= n_units) break;
-        const Unit w = make_unit(P, u);
         if (w.t[0].n == 0 && w.t[1].n == 0) continue;
         // (selects on scalars only: an index that depends on the warp would put the unit in
         // local memory)
@@ -738,9 +749,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       uint32_t qi = 0;                   // Q tiles of both streams so far (ring position)
       for (uint32_t kq = 0;; ++kq) {
         int u;
-        if (!next_unit(kq, u)) return;
+        Unit w;
+        if (!next_unit(kq, u, w)) return;
         if (u >= n_units) break;
-        const Unit w = make_unit(P, u);
         const QTile qt = s ? w.t[1] : w.t[0];
         const uint32_t my_qi = qi + ((s == 1 && w.t[0].n > 0) ? 1u : 0u);
         qi += (w.t[0].n > 0 ? 1u : 0u) + (w.t[1].n > 0 ? 1u : 0u);
