@@ -113,9 +113,26 @@ bool prefill_weights_supported(const Problem& P, const void* q, const void* k, c
 
 cudaError_t launch_prefill_weights(const Problem& P, const void* q, const void* k, const void* v, void* out,
                                    cudaStream_t stream, const char** msg) {
-  // 1. the forward, which also leaves each row's log-sum-exp in P.lse
-  cudaError_t e = launch_prefill(P, q, k, v, out, nullptr, stream, msg);
-  if (e != cudaSuccess) return e;
+  // 1. each row's log-sum-exp into P.lse (statistics only: the weights pass writes out)
+  prefill::TensorMaps maps{};
+  if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
+      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B)) {
+    if (msg) *msg = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
+  const int grid = (int)std::min<long long>(n_units, sm_count());
+  cudaError_t e;
+  if (P.dtype == SDPA_BF16)
+    e = P.D == 128 ? prefill::launch_stats<__nv_bfloat16, 128>(maps, P, out, grid, stream)
+                   : prefill::launch_stats<__nv_bfloat16, 64>(maps, P, out, grid, stream);
+  else
+    e = P.D == 128 ? prefill::launch_stats<__half, 128>(maps, P, out, grid, stream)
+                   : prefill::launch_stats<__half, 64>(maps, P, out, grid, stream);
+  if (e != cudaSuccess) {
+    if (msg) *msg = "statistics pass launch";
+    return e;
+  }
   // 2. the weights of the key tiles the weights pass does not visit
   const dim3 fgrid((unsigned)((P.Lq + prefill::kBlockM - 1) / prefill::kBlockM), (unsigned)P.H, (unsigned)P.B);
   if (P.dtype == SDPA_BF16)
@@ -128,14 +145,6 @@ cudaError_t launch_prefill_weights(const Problem& P, const void* q, const void* 
     return e;
   }
   // 3. the weights pass
-  prefill::TensorMaps maps{};
-  if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
-      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B)) {
-    if (msg) *msg = "cuTensorMapEncodeTiled failed";
-    return cudaErrorInvalidValue;
-  }
-  const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
-  const int grid = (int)std::min<long long>(n_units, sm_count());
   if (P.dtype == SDPA_BF16)
     e = P.D == 128 ? prefill::launch_weights<__nv_bfloat16, 128>(maps, P, out, grid, stream)
                    : prefill::launch_weights<__nv_bfloat16, 64>(maps, P, out, grid, stream);

@@ -83,8 +83,10 @@ enum { kMaskNone = 0, kMaskDense = 1, kMaskBits = 2 };
 // log-sum-exp when P.lse is set and the rotary embedding of the Q tiles when P.q_rope is set.
 // kModeWeights: scaled_dot_product_attention_with_weights given that log-sum-exp: the exact
 // weights 2^(x - lse) of the visited key tiles, dropped out and stored, and out = sum w' v.
-// (The plain forward carries none of the extra code.)
-enum { kModeForward = 0, kModeAux = 1, kModeWeights = 2 };
+// kModeStats: each row's log-sum-exp alone (P.lse; no bias or mask), for the weights pass that
+// follows: no V tiles, no PV, no output; the next S is issued as soon as the softmax has read
+// the current one. (The plain forward carries none of the extra code.)
+enum { kModeForward = 0, kModeAux = 1, kModeWeights = 2, kModeStats = 3 };
 
 // Shared-memory plan: the Q tiles of the two query tiles, the K and V rings, and with bias
 // tiles (kBT, head_dim 64) one bias tile per query tile. (A third Q slot, so that the next
@@ -489,7 +491,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                             kh, krow, kbt);
             }
           }
-          if (prev_kb >= 0) {
+          if (kMode != kModeStats && prev_kb >= 0) {
             const uint32_t x = g - 1;
             const int vs = x % C::kVStages;
             if (!wait_all(&v_empty[vs], ((x / C::kVStages) & 1) ^ 1)) return;
@@ -590,7 +592,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         // local memory)
         const int my_n = s == 0 ? w.t[0].n : w.t[1].n;
         const int n_o = s == 0 ? w.t[1].n : w.t[0].n;
-        const uint32_t groups_o = n_o > 0 ? (uint32_t)n_o + 1 : 0u;
+        // groups per tile: S(0); PV(j-1) + S(j); the last PV (statistics only: one per S)
+        const uint32_t groups_o = n_o > 0 ? (uint32_t)n_o + (kMode == kModeStats ? 0u : 1u) : 0u;
         // group k of this tile may be issued once the other tile has issued `before(k)` groups
         auto before = [&](uint32_t k) -> uint32_t { return base_o + min(s == 0 ? k : k + 1, groups_o); };
         // this tile's place in the Q ring: tile A, then tile B, of every unit with keys
@@ -673,7 +676,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             // a key tile only the other query tile visits: first the PV this tile owes (its
             // V slot may be needed before this warp reaches its next own key tile), then
             // release the slots once they hold this key tile
-            if (pend) {
+            if (kMode != kModeStats && pend) {
               if (!pv_ready(prev, first_pv)) return;
               if (!turn_wait(before(k_grp))) return;
               if (!pv(prev, first_pv, true)) return;
@@ -684,14 +687,21 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             }
             if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
             if (elected) mbar_arrive(&k_empty[ks]);
-            if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return;
-            if (elected) mbar_arrive(&v_empty[vs]);
+            if constexpr (kMode != kModeStats) {
+              if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return;
+              if (elected) mbar_arrive(&v_empty[vs]);
+            }
           } else {
             if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
-            if (pend && !pv_ready(prev, first_pv)) return;
+            if constexpr (kMode == kModeStats) {
+              // S(x) overwrites S(prev): the softmax has read it (it arrives on p_full then)
+              if (pend && !wait_all(&p_full[s], (sc - 1) & 1)) return;
+            } else {
+              if (pend && !pv_ready(prev, first_pv)) return;
+            }
             if (!turn_wait(before(k_grp))) return;
             // PV of this tile's previous key tile first: S(x) overwrites the P it reads
-            if (pend && !pv(prev, first_pv, false)) return;
+            if (kMode != kModeStats && pend && !pv(prev, first_pv, false)) return;
             if (pend) first_pv = false;
             tc_fence_after();
             if (elected) {
@@ -721,17 +731,22 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           if (nb == kb) ++jb;
           ++g;
         }
-        if (pend) {
-          if (!pv_ready(prev, first_pv)) return;
-          if (!turn_wait(before(k_grp))) return;
-          if (!pv(prev, first_pv, true)) return;
-          ++mine;
-          ++k_grp;
-        }
-        if (my_n > 0) {
-          if (elected) mma_commit(&o_ready[s]);
-          __syncwarp();
-          ++oc;
+        if constexpr (kMode == kModeStats) {
+          // the next unit's first S overwrites this unit's last one once the softmax has read it
+          if (pend && !wait_all(&p_full[s], (sc - 1) & 1)) return;
+        } else {
+          if (pend) {
+            if (!pv_ready(prev, first_pv)) return;
+            if (!turn_wait(before(k_grp))) return;
+            if (!pv(prev, first_pv, true)) return;
+            ++mine;
+            ++k_grp;
+          }
+          if (my_n > 0) {
+            if (elected) mma_commit(&o_ready[s]);
+            __syncwarp();
+            ++oc;
+          }
         }
         base_o += groups_o;
       }
@@ -778,9 +793,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
                                          (P.q_start ? (long long)P.Lq_total : (long long)P.B * P.Lq)));
         if (qt.n == 0) {
           // no key tile: NaN rows (nothing attended) or zero rows (past q_lengths)
-          if constexpr (kMode == kModeAux) {
+          if constexpr (kMode == kModeAux || kMode == kModeStats) {
             if (P.lse && i < P.Lq) P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = INFINITY;
           }
+          if constexpr (kMode == kModeStats) continue;  // the output is the weights pass's
           if (i < w.q_rows && row_ok) {
             const float val = (i >= w.q_len) ? 0.f : __int_as_float(0x7fc00000);
             const uint32_t wv = std::is_same<T, __half>::value ? pack_f16x2(val, val) : pack_bf16x2(val, val);
@@ -839,6 +855,12 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + scol + c * 32, v[c]);
           tmem_wait_ld();
+          if constexpr (kMode == kModeStats) {
+            // S is in registers: its columns are free for the next S
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[s]);
+          }
           if constexpr (kMode == kModeWeights) {
             // w = 2^(s * scale*log2e - lse) on the attended keys, 0 elsewhere, NaN for a row
             // with no key; the dropout keeps w / (1 - p) where the row's draw allows; the
@@ -1045,11 +1067,25 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
           const bool need_o = grow && had_max && j > 0;
           // O holds PV of the earlier key tiles (complete: the S commit covered them)
-          if (__any_sync(0xffffffffu, need_o)) rescale_o<D>(lane_addr + ocol, need_o ? alpha : 1.f);
+          if constexpr (kMode != kModeStats)
+            if (__any_sync(0xffffffffu, need_o)) rescale_o<D>(lane_addr + ocol, need_o ? alpha : 1.f);
           l *= alpha;
           const float negm = (m_used == -INFINITY) ? 0.f : -m_used;
           // P = 2^(v * mul - m), 16-bit pairs into the first 64 columns of the tile's S columns.
           float rs[4] = {0.f, 0.f, 0.f, 0.f};
+          if constexpr (kMode == kModeStats) {
+            // the row sum alone
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float x0, x1;
+                fma2(x0, x1, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), mul, mul, negm, negm);
+                add2(rs[(e >> 1) & 2], rs[((e >> 1) & 2) + 1], rs[(e >> 1) & 2], rs[((e >> 1) & 2) + 1], ex2(x0), ex2(x1));
+              }
+            l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            continue;
+          }
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[16];
@@ -1085,6 +1121,13 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[s]);
+        }
+        if constexpr (kMode == kModeStats) {
+          // the row's log-sum-exp in log2 units times lse_out_mul (+inf: no key, or padding)
+          if (i < P.Lq)
+            P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] =
+                (i < w.q_len && l > 0.f) ? (m_used + log2f(l)) * P.lse_out_mul : INFINITY;
+          continue;
         }
         if (!wait_all(&o_ready[s], oc & 1)) return;
         ++oc;
@@ -1172,6 +1215,13 @@ template <> cudaError_t launch_weights<__nv_bfloat16, 128>(const TensorMaps&, co
 template <> cudaError_t launch_weights<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
 template <> cudaError_t launch_weights<__half, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
 template <> cudaError_t launch_weights<__half, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+// Each row's log-sum-exp alone (kModeStats) into P.lse, for the weights pass
+template <typename T, int D>
+cudaError_t launch_stats(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream);
+template <> cudaError_t launch_stats<__nv_bfloat16, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_stats<__nv_bfloat16, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_stats<__half, 128>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
+template <> cudaError_t launch_stats<__half, 64>(const TensorMaps&, const Problem&, void*, int, cudaStream_t);
 
 // The weights of the key tiles a query tile does not visit (past its causal / kv_lengths bound,
 // the tiles make_qtile leaves out): 0, or NaN for a row with no key. Grid (query tiles, H, B);
@@ -1244,6 +1294,11 @@ inline int mask_variant(const Problem& P) {
   cudaError_t launch_weights<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,  \
                                    cudaStream_t stream) {                                           \
     return launch_variant<T, D, kBiasNone, kMaskNone, kModeWeights>(maps, P, out, grid, stream);   \
+  }                                                                                                 \
+  template <>                                                                                       \
+  cudaError_t launch_stats<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,    \
+                                 cudaStream_t stream) {                                             \
+    return launch_variant<T, D, kBiasNone, kMaskNone, kModeStats>(maps, P, out, grid, stream);     \
   }                                                                                                 \
   template <>                                                                                       \
   cudaError_t launch<T, D>(const TensorMaps& maps, const Problem& P, void* out, int grid,         \
