@@ -53,8 +53,15 @@ constexpr int kBlockN = 128;
 // soon as they are written (their PV steps start while the softmax finishes the rest), then the
 // remainder. (With head_dim 128 the split was measured 1-2% slower and P goes in one part.)
 constexpr int kEarlyKeys = 96;
-template <int D>
-constexpr bool kSplitP = D == 64;
+// With head_dim 64 and no bias the forward keeps P in TMEM columns of its own (384 + 64 *
+// stream: S and O take 384 of the 512): the next S is issued as soon as the softmax has read S,
+// and PV follows P, so the MMAs overlap the softmax instead of following it. (Measured: 3.5 %
+// faster without a bias, 8 % slower with the bias tiles, which keep P over S with the two-part
+// hand-over, as do the other modes.)
+template <int D, int kMode, int kBias>
+constexpr bool kSepP = D == 64 && (kMode == 0 || kMode == 1) && kBias == 0;
+template <int D, int kMode, int kBias>
+constexpr bool kSplitP = D == 64 && !kSepP<D, kMode, kBias>;
 constexpr int kThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer + MMA (+2 idle)
 // Register split (setmaxnreg): the two softmax warpgroups grow to kSoftmaxRegs, the last one
 // shrinks to kOtherRegs. 2*128*216 + 128*72 = 64512 = 384 * 168, the launch's registers; the
@@ -104,7 +111,7 @@ struct Cfg {
   static constexpr int kQSlots = 2;
   static constexpr int kBiasBytes = kBT ? 2 * kBiasSlots * kBiasTileBytes : 0;
   static constexpr int kBarriers =
-      3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots + 2;
+      3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots + 4;
   // tiles (+ the bias tiles), barriers, unit ring, TMEM address, abort flag, and slack to align
   // the base to 1024 bytes
   static constexpr int smem_bytes() {
@@ -327,8 +334,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint64_t* q_rot = drain + 1;                   // [kQSlots] Q tile rotated (P.q_rope)
   uint64_t* unit_full = q_rot + C::kQSlots;      // [kUnitSlots]
   uint64_t* unit_empty = unit_full + kUnitSlots; // [kUnitSlots]
-  uint64_t* p_early = unit_empty + kUnitSlots;  // [2] the first kEarlyKeys keys of P written
-  int* unit_ring = reinterpret_cast<int*>(p_early + 2);
+  // [2] the first kEarlyKeys keys of P written (kSepP: S read into the softmax's registers)
+  uint64_t* p_early = unit_empty + kUnitSlots;
+  uint64_t* p_free = p_early + 2;  // [2] kSepP: the PV of the stream's last P has completed
+  int* unit_ring = reinterpret_cast<int*>(p_free + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring + kUnitSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // MMA groups issued so far by the MMA warp of tile A / tile B (the turn order below)
@@ -349,6 +358,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4);  // one arrive per softmax warp
       mbar_init(&p_early[s], 4);
+      mbar_init(&p_free[s], 1);
       mbar_init(&o_ready[s], 1);
       mbar_init(&o_free[s], 4);
     }
@@ -593,7 +603,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         const int my_n = s == 0 ? w.t[0].n : w.t[1].n;
         const int n_o = s == 0 ? w.t[1].n : w.t[0].n;
         // groups per tile: S(0); PV(j-1) + S(j); the last PV (statistics only: one per S)
-        const uint32_t groups_o = n_o > 0 ? (uint32_t)n_o + (kMode == kModeStats ? 0u : 1u) : 0u;
+        const uint32_t groups_o =
+            n_o > 0 ? (uint32_t)n_o + ((kMode == kModeStats || kSepP<D, kMode, kBias>) ? 0u : 1u) : 0u;
         // group k of this tile may be issued once the other tile has issued `before(k)` groups
         auto before = [&](uint32_t k) -> uint32_t { return base_o + min(s == 0 ? k : k + 1, groups_o); };
         // this tile's place in the Q ring: tile A, then tile B, of every unit with keys
@@ -614,7 +625,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           const int vs = x % C::kVStages;
           if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
           if (first && !wait_all(&o_free[s], (oc & 1) ^ 1)) return false;
-          return wait_all(kSplitP<D> ? &p_early[s] : &p_full[s], (sc - 1) & 1);
+          return wait_all(kSplitP<D, kMode, kBias> ? &p_early[s] : &p_full[s], (sc - 1) & 1);
         };
         // O += P(x) V(x) for this tile's key tile at ring position x (after pv_ready): the steps
         // over the first kEarlyKeys keys, then, once the rest of P is written, the others (they
@@ -633,7 +644,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             }
           };
           tc_fence_after();
-          if constexpr (!kSplitP<D>) {
+          if constexpr (!kSplitP<D, kMode, kBias>) {
             if (elected) {
               steps(0, kBlockN / 16);
               if (last) publish();
@@ -661,6 +672,96 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
           return true;
         };
+        if constexpr (kSepP<D, kMode, kBias>) {
+          // P in its own columns: S(x) follows the softmax's read of S(prev) (turn order on the
+          // S groups), and PV(prev) follows P(prev), outside the turn order
+          const uint32_t p_tmem = tmem + 384 + s * 64;
+          int ja = 0, jb = 0, jm = 0;
+          uint32_t k_grp = 0;
+          bool s_pend = false, p_pend = false, first_pv = true;
+          uint32_t prev = 0, prev_si = 0;  // ring position and S index of this tile's last S
+          auto pv_sep = [&](uint32_t x, uint32_t si) -> bool {
+            const int vs = x % C::kVStages;
+            if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return false;
+            if (first_pv && !wait_all(&o_free[s], (oc & 1) ^ 1)) return false;
+            if (!wait_all(&p_full[s], si & 1)) return false;
+            tc_fence_after();
+            if (elected) {
+              const uint32_t vtile = v_base + vs * C::kTileBytes;
+#pragma unroll
+              for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                const uint64_t bdesc = smem_desc_sw128(vtile + kk * 16 * 128, kRegionBytes, 1024);
+                mma_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (first_pv && kk == 0) ? 0u : 1u);
+              }
+              mma_commit(&v_empty[vs]);
+              mma_commit(&p_free[s]);
+            }
+            __syncwarp();
+            first_pv = false;
+            return true;
+          };
+          for (;;) {
+            const int na = w.t[0].next(ja), nb = w.t[1].next(jb);
+            const int kb = min(na, nb);
+            if (kb == kNone) break;
+            const bool mine_tile = (s == 0 ? na : nb) == kb;
+            const uint32_t x = g;
+            const int ks = x % C::kKStages, vs = x % C::kVStages;
+            if (!mine_tile) {
+              // a key tile only the other query tile visits: the PV this tile owes, then release
+              // the slots once they hold this key tile
+              if (p_pend) {
+                if (!pv_sep(prev, prev_si)) return;
+                p_pend = false;
+              }
+              if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
+              if (elected) mbar_arrive(&k_empty[ks]);
+              if (!wait_all(&v_full[vs], (x / C::kVStages) & 1)) return;
+              if (elected) mbar_arrive(&v_empty[vs]);
+            } else {
+              if (!wait_all(&k_full[ks], (x / C::kKStages) & 1)) return;
+              // S(x) overwrites S(prev): the softmax has read it
+              if (s_pend && !wait_all(&p_early[s], prev_si & 1)) return;
+              if (!turn_wait(before(k_grp))) return;
+              tc_fence_after();
+              if (elected) {
+                const uint32_t ktile = k_base + ks * C::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = (kk / 4) * kRegionBytes + (kk % 4) * 32;
+                  mma_ss(s_tmem, smem_desc_sw128(qtile + off, 16, 1024), smem_desc_sw128(ktile + off, 16, 1024),
+                         idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                publish();
+                mma_commit(&s_full[s]);
+                mma_commit(&k_empty[ks]);
+                if (jm + 1 == my_n) mma_commit(&q_empty[qslot]);
+              }
+              __syncwarp();
+              ++mine;
+              ++k_grp;
+              const uint32_t si = sc++;
+              ++jm;
+              if (p_pend && !pv_sep(prev, prev_si)) return;
+              s_pend = p_pend = true;
+              prev = x;
+              prev_si = si;
+            }
+            if (na == kb) ++ja;
+            if (nb == kb) ++jb;
+            ++g;
+          }
+          if (p_pend && !pv_sep(prev, prev_si)) return;
+          // the next unit's first S overwrites this unit's last one once the softmax has read it
+          if (s_pend && !wait_all(&p_early[s], prev_si & 1)) return;
+          if (my_n > 0) {
+            if (elected) mma_commit(&o_ready[s]);
+            __syncwarp();
+            ++oc;
+          }
+          base_o += groups_o;
+          continue;
+        }
         int ja = 0, jb = 0, jm = 0;
         uint32_t k_grp = 0;  // groups of this tile issued in this unit
         bool pend = false, first_pv = true;
@@ -861,6 +962,12 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[s]);
           }
+          if constexpr (kSepP<D, kMode, kBias>) {
+            // S is in registers: its columns are free for the next S
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_early[s]);
+          }
           if constexpr (kMode == kModeWeights) {
             // w = 2^(s * scale*log2e - lse) on the attended keys, 0 elsewhere, NaN for a row
             // with no key; the dropout keeps w / (1 - p) where the row's draw allows; the
@@ -910,7 +1017,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-              if constexpr (kSplitP<D>) mbar_arrive(&p_early[s]);
+              if constexpr (kSplitP<D, kMode, kBias>) mbar_arrive(&p_early[s]);
               mbar_arrive(&p_full[s]);
             }
             continue;
@@ -1066,9 +1173,17 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             m_used = rmax;
           }
           const bool need_o = grow && had_max && j > 0;
-          // O holds PV of the earlier key tiles (complete: the S commit covered them)
-          if constexpr (kMode != kModeStats)
-            if (__any_sync(0xffffffffu, need_o)) rescale_o<D>(lane_addr + ocol, need_o ? alpha : 1.f);
+          // O holds PV of the earlier key tiles (complete: the S commit covered them; with P in
+          // its own columns the last PV is waited for here)
+          if constexpr (kMode != kModeStats) {
+            if (__any_sync(0xffffffffu, need_o)) {
+              if constexpr (kSepP<D, kMode, kBias>) {
+                if (!wait_all(&p_free[s], (sc - 2) & 1)) return;
+                tc_fence_after();
+              }
+              rescale_o<D>(lane_addr + ocol, need_o ? alpha : 1.f);
+            }
+          }
           l *= alpha;
           const float negm = (m_used == -INFINITY) ? 0.f : -m_used;
           // P = 2^(v * mul - m), 16-bit pairs into the first 64 columns of the tile's S columns.
@@ -1099,7 +1214,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             }
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[c / 2][(c % 2) * 16 + e] = pk[e];
-            if (kSplitP<D> && c == kEarlyKeys / 32 - 1) {
+            if (kSplitP<D, kMode, kBias> && c == kEarlyKeys / 32 - 1) {
               // keys [0, kEarlyKeys): 16-bit pairs in columns [0, kEarlyKeys / 2)
               static_assert(kEarlyKeys == 96, "P columns stored early: 32 + 16");
               tmem_st32(lane_addr + scol, v[0]);
@@ -1111,7 +1226,17 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             }
           }
           l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-          if constexpr (kSplitP<D>) {
+          if constexpr (kSepP<D, kMode, kBias>) {
+            // P's columns are free once the PV of this stream's last P has completed (the
+            // unit's first P follows the previous unit's output, which waited for all of them)
+            if (j > 0) {
+              if (!wait_all(&p_free[s], (sc - 2) & 1)) return;
+              tc_fence_after();
+            }
+            const uint32_t pcol = 384 + s * 64;
+            tmem_st32(lane_addr + pcol, v[0]);
+            tmem_st32(lane_addr + pcol + 32, v[1]);
+          } else if constexpr (kSplitP<D, kMode, kBias>) {
             tmem_st16(lane_addr + scol + kEarlyKeys / 2, *reinterpret_cast<const uint32_t(*)[16]>(&v[1][16]));
           } else {
             tmem_st32(lane_addr + scol, v[0]);
