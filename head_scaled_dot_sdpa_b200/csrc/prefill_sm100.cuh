@@ -268,10 +268,10 @@ __device__ __noinline__ void rescale_o(uint32_t taddr, float a) {
 
 // Rotary embedding of row r of a Q tile in shared memory (128-byte swizzle: logical 16-byte
 // chunk x of row r is stored at chunk x ^ (r % 8)): the pair (c, c + D/2) rotated by the angle
-// whose (cos, sin) fp16 pair is table[c]. Out of line, like rescale_o, so that the softmax
-// loop's code and registers stay as they are when no rotation is asked for.
+// whose (cos, sin) fp16 pair is table[c]. Inlined: it runs where the softmax's score registers
+// are not live (an out-of-line call saved and restored them around every rotation).
 template <typename T, int D>
-__device__ __noinline__ void rotate_q_row(uint8_t* tile, int r, const uint32_t* table) {
+__device__ __forceinline__ void rotate_q_row(uint8_t* tile, int r, const uint32_t* table) {
   constexpr int kHalf = D / 2, kPairChunks = kHalf / 8;
   const uint4* trow = reinterpret_cast<const uint4*>(table);
   uint4 tab[2 * kPairChunks];
