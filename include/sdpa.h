@@ -1,6 +1,7 @@
 /*
- * sdpa.h — C ABI of libsdpa.so: the forward pass of multi-head scaled-dot-product attention
- * on NVIDIA B200 (sm_100a).
+ * sdpa.h — C ABI of libsdpa.so: multi-head scaled-dot-product attention on NVIDIA B200
+ * (sm_100a): the forward pass, KV-cache decode, the gradient, the with-weights variant with
+ * dropout, and the rotary embedding of query / key rows.
  *
  * The operation is NNlib.scaled_dot_product_attention as the Flux.jl page "Neural Network
  * primitives from NNlib.jl" defines it (entry "scaled_dot_product_attention", section
@@ -228,8 +229,8 @@ SDPA_API sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed
  *  - The workspace holds the status word and one float per query row (the row's log-sum-exp):
  *    sdpa_weights_workspace_size(p) bytes.
  *  - Kernels. bf16/fp16 with dqk = dv = 64 or 128, no bias, mask or block_info, kv_len a
- *    multiple of 8 and 16-byte aligned arrays run on the tcgen05 prefill kernel: the forward
- *    (writing the row log-sum-exp), a kernel that writes the weights of the key tiles beyond
+ *    multiple of 8 and 16-byte aligned arrays run on the tcgen05 prefill kernel: a statistics
+ *    pass (the row log-sum-exp alone), a kernel that writes the weights of the key tiles beyond
  *    each query tile's causal / kv_lengths bound (0, or NaN for a row with no key), then the
  *    weights pass, which recomputes the logits on the tensor cores, stores the weights of the
  *    visited tiles with 16-byte stores and accumulates out from the dropped weights. Other
