@@ -162,7 +162,7 @@ cudaError_t launch_prefill(const Problem& P, const void* q, const void* k, const
   const bool packed = P.q_start != nullptr;
   const int q_rows = packed ? P.Lq_total : P.Lq, kv_rows = packed ? P.Lk_total : P.Lk, nb = packed ? 1 : P.B;
   if (!make_map(&maps.q, q, P.dtype, P.D, P.H, q_rows, nb) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, kv_rows, nb) ||
-      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, kv_rows, nb)) {
+      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, kv_rows, nb) || !make_map(&maps.o, out, P.dtype, P.D, P.H, q_rows, nb)) {
     if (msg) *msg = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }

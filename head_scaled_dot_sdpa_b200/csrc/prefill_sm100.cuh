@@ -62,6 +62,10 @@ template <int D, int kMode, int kBias>
 constexpr bool kSepP = D == 64 && (kMode == 0 || kMode == 1) && kBias == 0;
 template <int D, int kMode, int kBias>
 constexpr bool kSplitP = D == 64 && !kSepP<D, kMode, kBias>;
+// With head_dim 128 the forward writes O through a shared-memory staging tile and TMA stores
+// (one per 64-dim half), so that the stores are whole lines and leave the softmax warps at once.
+template <int D, int kMode>
+constexpr bool kOStage = D == 128 && (kMode == 0 || kMode == 1);
 constexpr int kThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer + MMA (+2 idle)
 // Register split (setmaxnreg): the two softmax warpgroups grow to kSoftmaxRegs, the last one
 // shrinks to kOtherRegs. 2*128*216 + 128*72 = 64512 = 384 * 168, the launch's registers; the
@@ -110,20 +114,23 @@ struct Cfg {
   // Q tiles: a ring shared by the two query tiles of the units, in the order A, B, A, B, ...
   static constexpr int kQSlots = 2;
   static constexpr int kBiasBytes = kBT ? 2 * kBiasSlots * kBiasTileBytes : 0;
+  // O staging (kOStage): one 128-row x 64-dim tile per query tile
+  static constexpr int kOStageBytes = 2 * 128 * 128;
   static constexpr int kBarriers =
-      3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots + 4;
+      3 * kQSlots + 2 * kKStages + 2 * kVStages + 2 * 4 + 2 * 2 * kBiasSlots + 1 + 2 * kUnitSlots + 8;
   // tiles (+ the bias tiles), barriers, unit ring, TMEM address, abort flag, and slack to align
   // the base to 1024 bytes
-  static constexpr int smem_bytes() {
-    return (kQSlots + kKStages + kVStages) * kTileBytes + kBiasBytes + kBarriers * 8 + 64 +
-           kUnitSlots * kUnitInfoBytes + 16 + 1024;
+  static constexpr int smem_bytes(bool ostage = false) {
+    return (kQSlots + kKStages + kVStages) * kTileBytes + kBiasBytes + (ostage ? kOStageBytes : 0) + kBarriers * 8 +
+           64 + kUnitSlots * kUnitInfoBytes + 16 + 1024;
   }
 };
 static_assert(Cfg<64, true>::smem_bytes() <= 227 * 1024, "bias tiles fit for head_dim 64");
-static_assert(Cfg<128>::smem_bytes() <= 227 * 1024 && Cfg<64>::smem_bytes() <= 227 * 1024, "tiles fit");
+static_assert(Cfg<128>::smem_bytes(true) <= 227 * 1024 && Cfg<64>::smem_bytes() <= 227 * 1024, "tiles fit");
 
 struct TensorMaps {
   CUtensorMap q, k, v, bias;  // bias: (keys, queries, heads, batch), used by kBiasTile only
+  CUtensorMap o;              // out, as q (the staged epilogue's stores)
 };
 
 // One query tile of a unit.
@@ -317,7 +324,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint8_t* k_smem = q_smem + C::kQSlots * C::kTileBytes;
   uint8_t* v_smem = k_smem + C::kKStages * C::kTileBytes;
   uint8_t* b_smem = v_smem + C::kVStages * C::kTileBytes;  // [2][kBiasSlots] bias tiles (kBiasTile)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + C::kBiasBytes);
+  uint8_t* o_stage = b_smem + C::kBiasBytes;  // [2] O staging tiles (kOStage)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(o_stage + (kOStage<D, kMode> ? C::kOStageBytes : 0));
   uint64_t* q_full = bars;                  // [kQSlots]
   uint64_t* q_empty = q_full + C::kQSlots;  // [kQSlots]
   uint64_t* k_full = q_empty + C::kQSlots;  // [KS]
@@ -337,7 +345,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   // [2] the first kEarlyKeys keys of P written (kSepP: S read into the softmax's registers)
   uint64_t* p_early = unit_empty + kUnitSlots;
   uint64_t* p_free = p_early + 2;  // [2] kSepP: the PV of the stream's last P has completed
-  int* unit_ring = reinterpret_cast<int*>(p_free + 2);
+  uint64_t* stage_free = p_free + 2;      // [2] kOStage: the stream's staging tile may be rewritten
+  uint64_t* stage_full = stage_free + 2;  // [2] kOStage: the staging tile is written
+  int* unit_ring = reinterpret_cast<int*>(stage_full + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring + kUnitSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // MMA groups issued so far by the MMA warp of tile A / tile B (the turn order below)
@@ -359,6 +369,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       mbar_init(&p_full[s], 4);  // one arrive per softmax warp
       mbar_init(&p_early[s], 4);
       mbar_init(&p_free[s], 1);
+      mbar_init(&stage_free[s], 1);  // the stream's leader thread, once the last store has read it
+      mbar_init(&stage_full[s], 4);  // one arrive per softmax warp
       mbar_init(&o_ready[s], 1);
       mbar_init(&o_free[s], 4);
     }
@@ -862,6 +874,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
       uint32_t sc = 0, oc = 0, bcs = 0;  // S tiles, units, bias tiles seen
+      uint32_t stg_n = 0;                // O staging halves written (kOStage)
       uint32_t qi = 0;                   // Q tiles of both streams so far (ring position)
       for (uint32_t kq = 0;; ++kq) {
         int u;
@@ -1265,6 +1278,56 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] =
                 (!pad && l > 0.f) ? (m_used + log2f(l)) * P.lse_out_mul : INFINITY;
         }
+        bool staged = false;
+        if constexpr (kOStage<D, kMode>) staged = P.q_start == nullptr;
+        if (staged) {
+          // Per 64-dim half: once the stream's staging tile is free (the leader thread's last
+          // store has read it), each thread writes its row, scaled and rounded, in the 128-byte
+          // swizzle (16-byte chunk x of row r at x ^ (r % 8)); the leader then stores the tile
+          // with TMA, which leaves out rows past the tensor unwritten.
+          uint8_t* stg = o_stage + s * (C::kOStageBytes / 2);
+          const bool leader = (threadIdx.x % 128) == 0;
+#pragma unroll 1
+          for (int hh = 0; hh < D / 64; ++hh) {
+            if (leader) {
+              bulk_wait_read();
+              mbar_arrive(&stage_free[s]);
+            }
+            if (!wait_all(&stage_free[s], stg_n & 1)) return;
+            uint32_t o[2][32];
+            tmem_ld32(lane_addr + ocol + hh * 64, o[0]);
+            tmem_ld32(lane_addr + ocol + hh * 64 + 32, o[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              uint32_t wv[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t* ox = &o[x / 4][(x % 4) * 8];
+                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(ox[2 * k]) * inv : inv);
+                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(ox[2 * k + 1]) * inv : inv);
+                wv[k] = std::is_same<T, __half>::value ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
+              }
+              *reinterpret_cast<uint4*>(stg + r * 128 + ((x ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&stage_full[s]);
+            if (warp % 4 == 0) {
+              if (!wait_all(&stage_full[s], stg_n & 1)) return;
+              if (leader) {
+                int oh = qt.h, orow0 = w.tq + qt.i0, ob = w.tb;
+                // range-checked build: a tile outside out is reported and not stored
+                if (SDPA_CHECKED(P.status, oh < P.H && orow0 < P.Lq && ob < P.B)) {
+                  tma_store_4d(&maps.o, stg, hh * 64, oh, orow0, ob);
+                  bulk_commit();
+                }
+              }
+              __syncwarp();
+            }
+            ++stg_n;
+          }
+        } else
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -1289,6 +1352,11 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if (lane == 0) mbar_arrive(&o_free[s]);
       }
     }();
+    // the staged output stores complete (their shared-memory source lives until then), also
+    // when the role ended on a timeout
+    if constexpr (kOStage<D, kMode>) {
+      if (threadIdx.x % 128 == 0) bulk_wait();
+    }
   }
   if (warp == kMmaWarpA || warp == kMmaWarpB) {
     // every MMA this CTA issued has completed before its TMEM is released (also on a timeout)
@@ -1376,7 +1444,7 @@ __global__ void __launch_bounds__(256) weights_fill_kernel(const Problem P) {
 template <typename T, int D, int kBias, int kMask, int kMode = kModeForward>
 cudaError_t launch_variant(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream) {
   auto kern = prefill_kernel<T, D, kBias, kMask, kMode>;
-  const int smem = Cfg<D, kBias == kBiasTile>::smem_bytes();
+  const int smem = Cfg<D, kBias == kBiasTile>::smem_bytes(kOStage<D, kMode>);
   // checked and configured once per device (bit d of `ready`)
   static std::atomic<unsigned long long> ready{0};
   int dev = 0;

@@ -80,6 +80,19 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const void* tmap, int c0, int
                "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                : "memory");
 }
+// Tile store from shared memory through a tensor map (no multicast), completed as a bulk
+// group of the issuing thread: bulk_commit() closes the group; bulk_wait_read() waits until
+// every committed group has finished reading shared memory, bulk_wait() until the writes are
+// done. Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const void* tmap, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
