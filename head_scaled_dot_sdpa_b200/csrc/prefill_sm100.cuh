@@ -874,7 +874,6 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
       uint32_t sc = 0, oc = 0, bcs = 0;  // S tiles, units, bias tiles seen
-      uint32_t stg_n = 0;                // O staging halves written (kOStage)
       uint32_t qi = 0;                   // Q tiles of both streams so far (ring position)
       for (uint32_t kq = 0;; ++kq) {
         int u;
@@ -1293,28 +1292,31 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               bulk_wait_read();
               mbar_arrive(&stage_free[s]);
             }
-            if (!wait_all(&stage_free[s], stg_n & 1)) return;
-            uint32_t o[2][32];
-            tmem_ld32(lane_addr + ocol + hh * 64, o[0]);
-            tmem_ld32(lane_addr + ocol + hh * 64 + 32, o[1]);
-            tmem_wait_ld();
+            // (two halves per unit, in every unit of the launch: the phase of half hh is hh % 2)
+            if (!wait_all(&stage_free[s], hh & 1)) return;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-              uint32_t wv[4];
+            for (int cc = 0; cc < 2; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(lane_addr + ocol + hh * 64 + cc * 32, o);
+              tmem_wait_ld();
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint32_t* ox = &o[x / 4][(x % 4) * 8];
-                const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(ox[2 * k]) * inv : inv);
-                const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(ox[2 * k + 1]) * inv : inv);
-                wv[k] = std::is_same<T, __half>::value ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
+              for (int xx = 0; xx < 4; ++xx) {
+                const int x = 4 * cc + xx;  // 16-byte chunk of the row's 64 dims
+                uint32_t wv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float a0 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[8 * xx + 2 * k]) * inv : inv);
+                  const float a1 = pad ? 0.f : (l > 0.f ? __uint_as_float(o[8 * xx + 2 * k + 1]) * inv : inv);
+                  wv[k] = std::is_same<T, __half>::value ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
+                }
+                *reinterpret_cast<uint4*>(stg + r * 128 + ((x ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
               }
-              *reinterpret_cast<uint4*>(stg + r * 128 + ((x ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
             asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&stage_full[s]);
             if (warp % 4 == 0) {
-              if (!wait_all(&stage_full[s], stg_n & 1)) return;
+              if (!wait_all(&stage_full[s], hh & 1)) return;
               if (leader) {
                 int oh = qt.h, orow0 = w.tq + qt.i0, ob = w.tb;
                 // range-checked build: a tile outside out is reported and not stored
@@ -1325,7 +1327,6 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               }
               __syncwarp();
             }
-            ++stg_n;
           }
         } else
 #pragma unroll
