@@ -53,6 +53,9 @@ struct Problem {
   unsigned long long drop_seed;
   unsigned drop_thr;
   float inv_keep;
+  // the statistics pass also writes the zero weights of the key tiles past each query tile's
+  // causal bound (set only when no row can lack a key, so that none of them is NaN)
+  int stats_fill;
   // rotary embedding of the Q tiles in shared memory (sdpa_forward_rope): (cos, sin) of each
   // query row's angles as fp16 pairs, [B * Lq][D / 2] 32-bit words; null when not rotated
   const uint32_t* q_rope;

@@ -111,8 +111,30 @@ bool prefill_weights_supported(const Problem& P, const void* q, const void* k, c
          prefill_supported(P, q, k, v, out);
 }
 
-cudaError_t launch_prefill_weights(const Problem& P, const void* q, const void* k, const void* v, void* out,
+// The weights as a 4-d tensor map (keys, queries, heads, batch), box 64 keys x 128 queries: the
+// statistics pass stores its zero tile through it.
+bool make_weights_map(CUtensorMap* m, const Problem& P) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)P.Lk, (cuuint64_t)P.Lq, (cuuint64_t)P.H, (cuuint64_t)P.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)P.Lk * 2, (cuuint64_t)P.Lq * P.Lk * 2, (cuuint64_t)P.H * P.Lq * P.Lk * 2};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt = P.dtype == SDPA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(m, dt, 4, P.weights, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_prefill_weights(const Problem& P0, const void* q, const void* k, const void* v, void* out,
                                    cudaStream_t stream, const char** msg) {
+  // Every row has a key (so no weight is NaN) when no kv_lengths cut the keys and the causal
+  // bound lets row 0 see key 0: then the statistics pass also writes the zero weights of the
+  // key tiles past each query tile's bound, and the fill kernel is not needed.
+  Problem P = P0;
+  const bool rows_have_keys =
+      P.kv_lengths == nullptr && P.Lk > 0 &&
+      (P.causal == SDPA_CAUSAL_NONE || (P.causal == SDPA_CAUSAL_TOP_LEFT && P.q_offset == nullptr && P.q_offset_scalar >= 0) ||
+       (P.causal == SDPA_CAUSAL_BOTTOM_RIGHT && P.Lk >= P.Lq));
   // 1. each row's log-sum-exp into P.lse (statistics only: the weights pass writes out)
   prefill::TensorMaps maps{};
   if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
@@ -120,6 +142,7 @@ cudaError_t launch_prefill_weights(const Problem& P, const void* q, const void* 
     if (msg) *msg = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
+  P.stats_fill = rows_have_keys && make_weights_map(&maps.w, P) ? 1 : 0;
   const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
   const int grid = (int)std::min<long long>(n_units, sm_count());
   cudaError_t e;
@@ -133,16 +156,19 @@ cudaError_t launch_prefill_weights(const Problem& P, const void* q, const void* 
     if (msg) *msg = "statistics pass launch";
     return e;
   }
-  // 2. the weights of the key tiles the weights pass does not visit
-  const dim3 fgrid((unsigned)((P.Lq + prefill::kBlockM - 1) / prefill::kBlockM), (unsigned)P.H, (unsigned)P.B);
-  if (P.dtype == SDPA_BF16)
-    prefill::weights_fill_kernel<__nv_bfloat16><<<fgrid, 256, 0, stream>>>(P);
-  else
-    prefill::weights_fill_kernel<__half><<<fgrid, 256, 0, stream>>>(P);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    if (msg) *msg = "weights fill launch";
-    return e;
+  // 2. the weights of the key tiles the weights pass does not visit (unless the statistics pass
+  // wrote them)
+  if (!P.stats_fill) {
+    const dim3 fgrid((unsigned)((P.Lq + prefill::kBlockM - 1) / prefill::kBlockM), (unsigned)P.H, (unsigned)P.B);
+    if (P.dtype == SDPA_BF16)
+      prefill::weights_fill_kernel<__nv_bfloat16><<<fgrid, 256, 0, stream>>>(P);
+    else
+      prefill::weights_fill_kernel<__half><<<fgrid, 256, 0, stream>>>(P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      if (msg) *msg = "weights fill launch";
+      return e;
+    }
   }
   // 3. the weights pass
   if (P.dtype == SDPA_BF16)

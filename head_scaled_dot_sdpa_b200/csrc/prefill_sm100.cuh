@@ -131,6 +131,7 @@ static_assert(Cfg<128>::smem_bytes(true) <= 227 * 1024 && Cfg<64>::smem_bytes() 
 struct TensorMaps {
   CUtensorMap q, k, v, bias;  // bias: (keys, queries, heads, batch), used by kBiasTile only
   CUtensorMap o;              // out, as q (the staged epilogue's stores)
+  CUtensorMap w;              // weights (keys, queries, heads, batch): the statistics pass's zero fill
 };
 
 // One query tile of a unit.
@@ -390,6 +391,14 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     issued[0] = 0;
     issued[1] = 0;
     fence_barrier_init();
+  }
+  if constexpr (kMode == kModeStats) {
+    // the zero tile of the weights fill: 64 keys x 128 rows, in the V ring (no V here)
+    if (P.stats_fill) {
+      for (int x = threadIdx.x; x < 128 * 128 / 16; x += blockDim.x)
+        reinterpret_cast<uint4*>(v_smem)[x] = make_uint4(0u, 0u, 0u, 0u);
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    }
   }
   if (warp == kMmaWarpA) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -874,6 +883,15 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
       uint32_t sc = 0, oc = 0, bcs = 0;  // S tiles, units, bias tiles seen
+      // statistics pass with the weights fill: the stream's leader stores the zero tile over the
+      // key tiles past the query tile's bound, 64 keys at a time (asynchronous TMA stores; the
+      // tensor map leaves out keys and rows past the array)
+      auto fill_zero_tail = [&](const Unit& uw, const QTile& uqt) {
+        if (threadIdx.x % 128 != 0) return;
+        const int nk64 = (P.Lk + 63) / 64;
+        for (int k2 = 2 * uqt.n; k2 < nk64; ++k2) tma_store_4d(&maps.w, v_smem, 64 * k2, uqt.i0, uqt.h, uw.b);
+        bulk_commit();
+      };
       uint32_t qi = 0;                   // Q tiles of both streams so far (ring position)
       for (uint32_t kq = 0;; ++kq) {
         int u;
@@ -909,7 +927,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           if constexpr (kMode == kModeAux || kMode == kModeStats) {
             if (P.lse && i < P.Lq) P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = INFINITY;
           }
-          if constexpr (kMode == kModeStats) continue;  // the output is the weights pass's
+          if constexpr (kMode == kModeStats) {
+            if (P.stats_fill && qt.i0 < P.Lq) fill_zero_tail(w, qt);
+            continue;  // the output is the weights pass's
+          }
           if (i < w.q_rows && row_ok) {
             const float val = (i >= w.q_len) ? 0.f : __int_as_float(0x7fc00000);
             const uint32_t wv = std::is_same<T, __half>::value ? pack_f16x2(val, val) : pack_bf16x2(val, val);
@@ -1264,6 +1285,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           if (i < P.Lq)
             P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] =
                 (i < w.q_len && l > 0.f) ? (m_used + log2f(l)) * P.lse_out_mul : INFINITY;
+          if (P.stats_fill) fill_zero_tail(w, qt);
           continue;
         }
         if (!wait_all(&o_ready[s], oc & 1)) return;
@@ -1355,7 +1377,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     }();
     // the staged output stores complete (their shared-memory source lives until then), also
     // when the role ended on a timeout
-    if constexpr (kOStage<D, kMode>) {
+    if constexpr (kOStage<D, kMode> || kMode == kModeStats) {
       if (threadIdx.x % 128 == 0) bulk_wait();
     }
   }
