@@ -111,14 +111,15 @@ bool prefill_weights_supported(const Problem& P, const void* q, const void* k, c
          prefill_supported(P, q, k, v, out);
 }
 
-// The weights as a 4-d tensor map (keys, queries, heads, batch), box 64 keys x 128 queries: the
-// statistics pass stores its zero tile through it.
-bool make_weights_map(CUtensorMap* m, const Problem& P) {
+// The weights as a 4-d tensor map (keys, queries, heads, batch), box 64 keys x `rows` queries in
+// the 128-byte swizzle: 128 rows for the statistics pass's zero tile, 32 for the weights pass's
+// stores (one warp's rows).
+bool make_weights_map(CUtensorMap* m, const Problem& P, unsigned rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)P.Lk, (cuuint64_t)P.Lq, (cuuint64_t)P.H, (cuuint64_t)P.B};
   const cuuint64_t strides[3] = {(cuuint64_t)P.Lk * 2, (cuuint64_t)P.Lq * P.Lk * 2, (cuuint64_t)P.H * P.Lq * P.Lk * 2};
-  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t box[4] = {64, rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapDataType dt = P.dtype == SDPA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   return fn(m, dt, 4, P.weights, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -138,11 +139,12 @@ cudaError_t launch_prefill_weights(const Problem& P0, const void* q, const void*
   // 1. each row's log-sum-exp into P.lse (statistics only: the weights pass writes out)
   prefill::TensorMaps maps{};
   if (!make_map(&maps.q, q, P.dtype, P.D, P.H, P.Lq, P.B) || !make_map(&maps.k, k, P.dtype, P.D, P.Hkv, P.Lk, P.B) ||
-      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B)) {
+      !make_map(&maps.v, v, P.dtype, P.D, P.Hkv, P.Lk, P.B) || !make_weights_map(&maps.w, P, 128) ||
+      !make_weights_map(&maps.w_warp, P, 32)) {
     if (msg) *msg = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
-  P.stats_fill = rows_have_keys && make_weights_map(&maps.w, P) ? 1 : 0;
+  P.stats_fill = rows_have_keys ? 1 : 0;
   const long long n_units = (long long)prefill::units_per_level(P) * prefill::n_levels(P);
   const int grid = (int)std::min<long long>(n_units, sm_count());
   cudaError_t e;

@@ -66,6 +66,10 @@ constexpr bool kSplitP = D == 64 && !kSepP<D, kMode, kBias>;
 // (one per 64-dim half), so that the stores are whole lines and leave the softmax warps at once.
 template <int D, int kMode>
 constexpr bool kOStage = D == 128 && (kMode == 0 || kMode == 1);
+// The weights pass stores its weight tiles through the same staging tiles (one 64-key half at a
+// time), with either head_dim.
+template <int D, int kMode>
+constexpr bool kStageSmem = kOStage<D, kMode> || kMode == 2;
 constexpr int kThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer + MMA (+2 idle)
 // Register split (setmaxnreg): the two softmax warpgroups grow to kSoftmaxRegs, the last one
 // shrinks to kOtherRegs. 2*128*216 + 128*72 = 64512 = 384 * 168, the launch's registers; the
@@ -131,7 +135,8 @@ static_assert(Cfg<128>::smem_bytes(true) <= 227 * 1024 && Cfg<64>::smem_bytes() 
 struct TensorMaps {
   CUtensorMap q, k, v, bias;  // bias: (keys, queries, heads, batch), used by kBiasTile only
   CUtensorMap o;              // out, as q (the staged epilogue's stores)
-  CUtensorMap w;              // weights (keys, queries, heads, batch): the statistics pass's zero fill
+  CUtensorMap w;              // weights (keys, queries, heads, batch), box 64 x 128: the zero fill
+  CUtensorMap w_warp;         // the same, box 64 keys x 32 rows: one warp's staged weights
 };
 
 // One query tile of a unit.
@@ -325,8 +330,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
   uint8_t* k_smem = q_smem + C::kQSlots * C::kTileBytes;
   uint8_t* v_smem = k_smem + C::kKStages * C::kTileBytes;
   uint8_t* b_smem = v_smem + C::kVStages * C::kTileBytes;  // [2][kBiasSlots] bias tiles (kBiasTile)
-  uint8_t* o_stage = b_smem + C::kBiasBytes;  // [2] O staging tiles (kOStage)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(o_stage + (kOStage<D, kMode> ? C::kOStageBytes : 0));
+  uint8_t* o_stage = b_smem + C::kBiasBytes;  // [2] staging tiles of O or of the weights (kStageSmem)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(o_stage + (kStageSmem<D, kMode> ? C::kOStageBytes : 0));
   uint64_t* q_full = bars;                  // [kQSlots]
   uint64_t* q_empty = q_full + C::kQSlots;  // [kQSlots]
   uint64_t* k_full = q_empty + C::kQSlots;  // [KS]
@@ -952,16 +957,14 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         if constexpr (kMask == kMaskDense)
           mask_row = P.mask + (long long)i * P.ms[1] + (long long)qt.h * P.ms[2] + (long long)w.b * P.ms[3];
         float m_used = -INFINITY, l = 0.f;
-        // weights pass: the row's log-sum-exp from the forward (+inf: no key, or padding), the
-        // row of the weights, and its first position (the dropout counter)
+        // weights pass: the row's log-sum-exp from the statistics pass (+inf: no key, or
+        // padding) and the row's first position in the weights (the dropout counter)
         float row_lse = INFINITY;
-        T* wrow = nullptr;
         unsigned long long wbase = 0;
         if constexpr (kMode == kModeWeights) {
           const long long wr = ((long long)w.b * P.H + qt.h) * P.Lq + i;
           if (i < P.Lq) {
             row_lse = P.lse[wr];
-            wrow = static_cast<T*>(P.weights) + wr * P.Lk;
             wbase = (unsigned long long)wr * (unsigned long long)P.Lk;
           }
           if (i < w.q_len && row_lse != INFINITY) l = 1.f;  // O is already normalised
@@ -1003,43 +1006,73 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
           if constexpr (kMode == kModeWeights) {
             // w = 2^(s * scale*log2e - lse) on the attended keys, 0 elsewhere, NaN for a row
-            // with no key; the dropout keeps w / (1 - p) where the row's draw allows; the
-            // weights go to global memory in 16-byte stores and w' into TMEM for the PV MMA
+            // with no key. Dropout: the weight takes 16-bit field u of its group's draw; with f
+            // the float 2^23 + u (u under the exponent bits of 2^23), sat(f + 1 - thr - 2^23) is
+            // exactly 1 when u >= thr (kept) and 0 otherwise, and the kept weight's 1/(1 - p) is
+            // in the exponent. Keys past the row's bound are zeroed after the 16-bit packing,
+            // on the tiles where a row of the warp has such keys. w' goes into TMEM for the PV
+            // MMA; the weights go through the warp's part of the staging tile to TMA stores.
             const bool nan_row = i < w.q_len && row_lse == INFINITY;
-            const float negl = nan_row ? 0.f : -row_lse;
-            const uint32_t nanw = std::is_same<T, __half>::value ? 0x7E007E00u : 0x7FC07FC0u;
+            const bool drop = P.drop_thr > 0;
+            const float negl = nan_row ? 0.f : -row_lse + (drop ? log2f(P.inv_keep) : 0.f);
+            const float kthr = 1.f - (float)P.drop_thr - 8388608.f;
+            // One 64-key half of the warp's 32 rows (v[hh]: this thread's row) in the 128-byte
+            // swizzle (16-byte chunk x of row r at x ^ (r % 8)), once the warp's previous store
+            // has read its 4 KB; lane 0 then stores it with TMA, which leaves out rows and keys
+            // past the array. Both halves go out after P is handed over, while the MMAs run.
+            uint8_t* stg = o_stage + s * (C::kOStageBytes / 2) + (warp % 4) * (32 * 128);
+            const int wrow0 = qt.i0 + 32 * (warp % 4);
+            auto stage_half = [&](int hh) {
+              if (lane == 0) bulk_wait_read();
+              __syncwarp();
+              const uint32_t nanw = std::is_same<T, __half>::value ? 0x7E007E00u : 0x7FC07FC0u;
+#pragma unroll
+              for (int x = 0; x < 8; ++x) {
+                const uint4 st = nan_row ? make_uint4(nanw, nanw, nanw, nanw)
+                                         : make_uint4(v[hh][4 * x], v[hh][4 * x + 1], v[hh][4 * x + 2], v[hh][4 * x + 3]);
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((x ^ (lane & 7)) << 4)) = st;
+              }
+              asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+              __syncwarp();
+              // range-checked build: a half outside the weights is reported and not stored
+              if (lane == 0 && key0 + 64 * hh < P.Lk && wrow0 < P.Lq &&
+                  SDPA_CHECKED(P.status, qt.h < P.H && w.b < P.B)) {
+                tma_store_4d(&maps.w_warp, stg, key0 + 64 * hh, wrow0, qt.h, w.b);
+                bulk_commit();
+              }
+            };
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               const int lim = nvalid - 32 * c;
-              uint32_t keep = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
-              if (P.drop_thr > 0) {
-                uint32_t kd = 0;
-                // the 8 groups of these 32 keys: consecutive draws, one gamma apart
-                unsigned long long z = dropout_state(P.drop_seed, (wbase + (unsigned long long)(key0 + 32 * c)) >> 2);
-#pragma unroll
-                for (int gq = 0; gq < 8; ++gq, z += kSplitMixGamma)
-                  kd |= dropout_keep4(splitmix64_mix(z), P.drop_thr) << (4 * gq);
-                keep &= kd;
-              }
-              const float sc_keep = P.drop_thr > 0 ? P.inv_keep : 1.f;
+              // the 8 groups of these 32 keys: consecutive draws, one gamma apart in the state
+              unsigned long long z = drop ? dropout_state(P.drop_seed, (wbase + (unsigned long long)(key0 + 32 * c)) >> 2) : 0ull;
               uint32_t pk[16];
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                float x0, x1;
-                fma2(x0, x1, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), sl2, sl2, negl, negl);
-                const float p0 = ((keep >> e) & 1u) ? ex2(x0) * sc_keep : 0.f;
-                const float p1 = ((keep >> (e + 1)) & 1u) ? ex2(x1) * sc_keep : 0.f;
-                pk[e / 2] = std::is_same<T, __half>::value ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
-              }
-              if (wrow) {
-#pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                  // 8 weights (kv_len is a multiple of 8, so a run is inside the row or past it)
-                  if (key0 + 32 * c + 2 * e < P.Lk) {
-                    const uint4 st = nan_row ? make_uint4(nanw, nanw, nanw, nanw) : make_uint4(pk[e], pk[e + 1], pk[e + 2], pk[e + 3]);
-                    *reinterpret_cast<uint4*>(wrow + key0 + 32 * c + 2 * e) = st;
-                  }
+              for (int gq = 0; gq < 8; ++gq) {
+                float mk[4] = {1.f, 1.f, 1.f, 1.f};
+                if (drop) {
+                  const unsigned long long rr = splitmix64_mix(z);
+                  z += kSplitMixGamma;
+                  const uint32_t lo = (uint32_t)rr, hi = (uint32_t)(rr >> 32);
+                  mk[0] = __saturatef(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7610)) + kthr);
+                  mk[1] = __saturatef(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7632)) + kthr);
+                  mk[2] = __saturatef(__uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7610)) + kthr);
+                  mk[3] = __saturatef(__uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7632)) + kthr);
                 }
+                const int e = 4 * gq;
+                float x0, x1, x2, x3;
+                fma2(x0, x1, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]), sl2, sl2, negl, negl);
+                fma2(x2, x3, __uint_as_float(v[c][e + 2]), __uint_as_float(v[c][e + 3]), sl2, sl2, negl, negl);
+                const float p0 = ex2(x0) * mk[0], p1 = ex2(x1) * mk[1], p2 = ex2(x2) * mk[2], p3 = ex2(x3) * mk[3];
+                pk[2 * gq] = std::is_same<T, __half>::value ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+                pk[2 * gq + 1] = std::is_same<T, __half>::value ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
+              }
+              if (__any_sync(0xffffffffu, lim < 32)) {
+                // keys [lim, 32) of this chunk are past the row's bound (their exponentials
+                // may be anything): the pair (2e, 2e + 1) keeps what lies below lim
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                  pk[e] = 2 * e + 1 < lim ? pk[e] : (2 * e < lim ? (pk[e] & 0xFFFFu) : 0u);
               }
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[c / 2][(c % 2) * 16 + e] = pk[e];
@@ -1053,6 +1086,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
               if constexpr (kSplitP<D, kMode, kBias>) mbar_arrive(&p_early[s]);
               mbar_arrive(&p_full[s]);
             }
+            stage_half(0);
+            stage_half(1);
             continue;
           }
           // Fast path (no bias, no mask bytes, every key of the tile attended by every row of
@@ -1377,8 +1412,8 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
     }();
     // the staged output stores complete (their shared-memory source lives until then), also
     // when the role ended on a timeout
-    if constexpr (kOStage<D, kMode> || kMode == kModeStats) {
-      if (threadIdx.x % 128 == 0) bulk_wait();
+    if constexpr (kStageSmem<D, kMode> || kMode == kModeStats) {
+      if (threadIdx.x % 128 == 0 || (kMode == kModeWeights && lane == 0)) bulk_wait();
     }
   }
   if (warp == kMmaWarpA || warp == kMmaWarpB) {
@@ -1467,7 +1502,7 @@ __global__ void __launch_bounds__(256) weights_fill_kernel(const Problem P) {
 template <typename T, int D, int kBias, int kMask, int kMode = kModeForward>
 cudaError_t launch_variant(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream) {
   auto kern = prefill_kernel<T, D, kBias, kMask, kMode>;
-  const int smem = Cfg<D, kBias == kBiasTile>::smem_bytes(kOStage<D, kMode>);
+  const int smem = Cfg<D, kBias == kBiasTile>::smem_bytes(kStageSmem<D, kMode>);
   // checked and configured once per device (bit d of `ready`)
   static std::atomic<unsigned long long> ready{0};
   int dev = 0;
