@@ -66,8 +66,8 @@ constexpr bool kSplitP = D == 64 && !kSepP<D, kMode, kBias>;
 // (one per 64-dim half), so that the stores are whole lines and leave the softmax warps at once.
 template <int D, int kMode>
 constexpr bool kOStage = D == 128 && (kMode == 0 || kMode == 1);
-// The weights pass stores its weight tiles through the same staging tiles (one 64-key half at a
-// time), with either head_dim.
+// The weights pass stores its weight tiles through the same staging tiles (each softmax warp its
+// 32 rows, one 64-key half at a time), with either head_dim.
 template <int D, int kMode>
 constexpr bool kStageSmem = kOStage<D, kMode> || kMode == 2;
 constexpr int kThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer + MMA (+2 idle)
@@ -888,13 +888,25 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
       uint32_t sc = 0, oc = 0, bcs = 0;  // S tiles, units, bias tiles seen
-      // statistics pass with the weights fill: the stream's leader stores the zero tile over the
-      // key tiles past the query tile's bound, 64 keys at a time (asynchronous TMA stores; the
-      // tensor map leaves out keys and rows past the array)
+      // Statistics pass with the weights fill: after query tile t of a (batch, head), the
+      // stream's leader stores the zero tile over the key tiles past the bound of the mirror
+      // tile nqt - 1 - t of the same (batch, head), 64 keys at a time (asynchronous TMA stores;
+      // the tensor map leaves out keys and rows past the array). Every tile is visited once, so
+      // every tile's zeros are written once; mirrored, the largest fills (short causal rows) ride
+      // with the longest rows, which run first, instead of piling up at the end of the launch.
       auto fill_zero_tail = [&](const Unit& uw, const QTile& uqt) {
         if (threadIdx.x % 128 != 0) return;
+        BatchInfo bi;
+        bi.q_len = uw.q_len;
+        bi.kv_len = uw.kv_len;
+        bi.offset = uw.offset;
+        bi.skip = false;
+        bi.q_rows = uw.q_rows;
+        bi.q0 = bi.k0 = 0;
+        const int nqt = (P.Lq + kBlockM - 1) / kBlockM;
+        const QTile mq = make_qtile(P, bi, uqt.h, nqt - 1 - uqt.qt, true);
         const int nk64 = (P.Lk + 63) / 64;
-        for (int k2 = 2 * uqt.n; k2 < nk64; ++k2) tma_store_4d(&maps.w, v_smem, 64 * k2, uqt.i0, uqt.h, uw.b);
+        for (int k2 = 2 * mq.n; k2 < nk64; ++k2) tma_store_4d(&maps.w, v_smem, 64 * k2, mq.i0, mq.h, uw.b);
         bulk_commit();
       };
       uint32_t qi = 0;                   // Q tiles of both streams so far (ring position)
@@ -1450,8 +1462,9 @@ template <> cudaError_t launch<__nv_bfloat16, 64>(const TensorMaps&, const Probl
 template <> cudaError_t launch<__half, 128>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
 template <> cudaError_t launch<__half, 64>(const TensorMaps&, const Problem&, void*, int, bool, cudaStream_t);
 
-// The weights pass (kModeWeights, no bias or mask) for one (T, D) pair, after the forward has
-// written P.lse and weights_fill_kernel the key tiles the pass does not visit.
+// The weights pass (kModeWeights, no bias or mask) for one (T, D) pair, after the statistics pass
+// has written P.lse and the weights of the key tiles the pass does not visit have been written
+// (by the statistics pass or weights_fill_kernel).
 template <typename T, int D>
 cudaError_t launch_weights(const TensorMaps& maps, const Problem& P, void* out, int grid, cudaStream_t stream);
 // The forward with the row log-sum-exp (P.lse) and / or the rotated Q tiles (P.q_rope); no bias
