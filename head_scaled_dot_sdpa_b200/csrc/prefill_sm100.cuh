@@ -888,13 +888,15 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
       const uint32_t scol = s * 128, ocol = 256 + s * D;
       const float sl2 = P.scale_log2;
       uint32_t sc = 0, oc = 0, bcs = 0;  // S tiles, units, bias tiles seen
-      // Statistics pass with the weights fill: after query tile t of a (batch, head), the
-      // stream's leader stores the zero tile over the key tiles past the bound of the mirror
-      // tile nqt - 1 - t of the same (batch, head), 64 keys at a time (asynchronous TMA stores;
-      // the tensor map leaves out keys and rows past the array). Every tile is visited once, so
-      // every tile's zeros are written once; mirrored, the largest fills (short causal rows) ride
-      // with the longest rows, which run first, instead of piling up at the end of the launch.
-      auto fill_zero_tail = [&](const Unit& uw, const QTile& uqt) {
+      // Statistics pass with the weights fill: while query tile t of a (batch, head) is
+      // processed, the stream's leader stores the zero tile over the key tiles past the bound of
+      // the mirror tile nqt - 1 - t of the same (batch, head), 64 keys per TMA store (the tensor
+      // map leaves out keys and rows past the array), a share after each key tile so that the
+      // stores do not hold up the K loads in the TMA unit. Every tile is visited once, so every
+      // tile's zeros are written once; mirrored, the largest fills (short causal rows) ride with
+      // the longest rows, which run first, instead of piling up at the end of the launch.
+      int fz_next = 0, fz_end = 0, fz_per = 0, fz_i0 = 0, fz_h = 0, fz_b = 0;
+      auto fill_begin = [&](const Unit& uw, const QTile& uqt) {
         if (threadIdx.x % 128 != 0) return;
         BatchInfo bi;
         bi.q_len = uw.q_len;
@@ -905,8 +907,17 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
         bi.q0 = bi.k0 = 0;
         const int nqt = (P.Lq + kBlockM - 1) / kBlockM;
         const QTile mq = make_qtile(P, bi, uqt.h, nqt - 1 - uqt.qt, true);
-        const int nk64 = (P.Lk + 63) / 64;
-        for (int k2 = 2 * mq.n; k2 < nk64; ++k2) tma_store_4d(&maps.w, v_smem, 64 * k2, mq.i0, mq.h, uw.b);
+        fz_next = 2 * mq.n;
+        fz_end = max((P.Lk + 63) / 64, fz_next);
+        fz_per = uqt.n > 0 ? (fz_end - fz_next + uqt.n - 1) / uqt.n : fz_end - fz_next;
+        fz_i0 = mq.i0;
+        fz_h = mq.h;
+        fz_b = uw.b;
+      };
+      auto fill_some = [&](int count) {
+        if (threadIdx.x % 128 != 0 || fz_next >= fz_end) return;
+        for (int x = 0; x < count && fz_next < fz_end; ++x, ++fz_next)
+          tma_store_4d(&maps.w, v_smem, 64 * fz_next, fz_i0, fz_h, fz_b);
         bulk_commit();
       };
       uint32_t qi = 0;                   // Q tiles of both streams so far (ring position)
@@ -945,7 +956,10 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             if (P.lse && i < P.Lq) P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] = INFINITY;
           }
           if constexpr (kMode == kModeStats) {
-            if (P.stats_fill && qt.i0 < P.Lq) fill_zero_tail(w, qt);
+            if (P.stats_fill && qt.i0 < P.Lq) {
+              fill_begin(w, qt);
+              fill_some(fz_per);
+            }
             continue;  // the output is the weights pass's
           }
           if (i < w.q_rows && row_ok) {
@@ -981,6 +995,9 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           }
           if (i < w.q_len && row_lse != INFINITY) l = 1.f;  // O is already normalised
         }
+        if constexpr (kMode == kModeStats) {
+          if (P.stats_fill) fill_begin(w, qt);
+        }
         for (int j = 0; j < qt.n; ++j) {
           const int kb = qt.kb(j);
           const int key0 = kb * kBlockN;
@@ -1009,6 +1026,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[s]);
+            if (P.stats_fill) fill_some(fz_per);
           }
           if constexpr (kSepP<D, kMode, kBias>) {
             // S is in registers: its columns are free for the next S
@@ -1332,7 +1350,7 @@ prefill_kernel(const __grid_constant__ TensorMaps maps, const Problem P, T* __re
           if (i < P.Lq)
             P.lse[((long long)w.b * P.H + qt.h) * P.Lq + i] =
                 (i < w.q_len && l > 0.f) ? (m_used + log2f(l)) * P.lse_out_mul : INFINITY;
-          if (P.stats_fill) fill_zero_tail(w, qt);
+          if (P.stats_fill) fill_some(fz_end);
           continue;
         }
         if (!wait_all(&o_ready[s], oc & 1)) return;
