@@ -230,10 +230,11 @@ SDPA_API sdpa_status sdpa_forward_packed(const sdpa_params* p, const sdpa_packed
  *    sdpa_weights_workspace_size(p) bytes.
  *  - Kernels. bf16/fp16 with dqk = dv = 64 or 128, no bias, mask or block_info, kv_len a
  *    multiple of 8 and 16-byte aligned arrays run on the tcgen05 prefill kernel: a statistics
- *    pass (the row log-sum-exp alone), a kernel that writes the weights of the key tiles beyond
- *    each query tile's causal / kv_lengths bound (0, or NaN for a row with no key), then the
- *    weights pass, which recomputes the logits on the tensor cores, stores the weights of the
- *    visited tiles with 16-byte stores and accumulates out from the dropped weights. Other
+ *    pass (the row log-sum-exp alone), the weights of the key tiles beyond each query tile's
+ *    causal / kv_lengths bound (0, or NaN for a row with no key: written by the statistics pass
+ *    when no row can be empty, else by a fill kernel), then the weights pass, which recomputes
+ *    the logits on the tensor cores, accumulates out from the dropped weights and stores the
+ *    weights of the visited tiles through shared memory with TMA. Other
  *    bf16/fp16 calls with dqk = dv = 64 or 128 take mma.sync tiles; a SIMT kernel handles the
  *    rest, or runs when SDPA_FLAG_GENERIC_KERNEL is set. */
 SDPA_API size_t sdpa_weights_workspace_size(const sdpa_params* p);
