@@ -65,6 +65,7 @@ SHAPES = [
     (2, 64, 33, 3, 3, 40, 24),
     (2, 150, 264, 8, 2, 64, 64),
     (1, 300, 384, 4, 4, 128, 128),
+    (1, 390, 136, 4, 2, 128, 128),  # more queries than keys, an odd number of query tiles
 ]
 
 
@@ -101,6 +102,17 @@ def test_weights_tcgen05_lengths_and_empty_rows(dtype):
           q_lengths=[200, 131, 12], kv_lengths=[264, 140, 0], drop_p=0.1, seed=5)
     check(q, k, v, "tcgen05 bottom right", kernel="weights_tcgen05", is_causal="bottom_right",
           q_lengths=[200, 131, 12], kv_lengths=[264, 140, 8], drop_p=0.3, seed=6)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_weights_tcgen05_scalar_offset_fill(dtype):
+    """Causal with a scalar q_offset >= 0 (every row sees key 0): the statistics pass writes the
+    zero weights past the causal bounds (query tile t writes those of tile nqt - 1 - t; three
+    query tiles, so the middle one is its own mirror), and the last key tile holds 8 keys."""
+    q, k, v = _inputs(21, 2, 300, 520, 4, 2, 128, 128, dtype)
+    check(q, k, v, "tcgen05 scalar offset", kernel="weights_tcgen05", is_causal=True, q_offset=40, drop_p=0.1,
+          seed=9)
+    check(q, k, v, "tcgen05 scalar offset, p = 0", kernel="weights_tcgen05", is_causal=True, q_offset=200)
 
 
 def test_weights_causal_gqa_workload_rows():
