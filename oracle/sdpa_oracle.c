@@ -350,12 +350,16 @@ int oracle_sdpa_backward(const oracle_sdpa_problem* p, const double* q, const do
   memset(dq, 0, sizeof(double) * (size_t)(B * Lq * H * D));
   memset(dk, 0, sizeof(double) * (size_t)(B * Lk * Hkv * D));
   memset(dv, 0, sizeof(double) * (size_t)(B * Lk * Hkv * Dv));
-  double total = 0.0;
   int failed = 0;
+  /* dscale's share of each (batch, key/value head), summed in that order after the loop, so
+   * that the result does not depend on how the threads took the units */
+  double* part = (double*)calloc((size_t)(B * Hkv > 0 ? B * Hkv : 1), sizeof(double));
+  if (!part) return ORACLE_ERR_NOMEM;
   /* each (batch, key/value head) owns its rows of dk and dv */
-#pragma omp parallel for schedule(dynamic, 1) reduction(+ : total)
+#pragma omp parallel for schedule(dynamic, 1)
   for (int64_t bg = 0; bg < B * Hkv; ++bg) {
     const int64_t b = bg / Hkv, g = bg % Hkv;
+    double total = 0.0;
     double* x = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
     double* dw = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
     unsigned char* ok = (unsigned char*)malloc((size_t)(Lk > 0 ? Lk : 1));
@@ -428,10 +432,14 @@ int oracle_sdpa_backward(const oracle_sdpa_problem* p, const double* q, const do
         }
       }
     }
+    part[bg] = total;
     free(x);
     free(dw);
     free(ok);
   }
+  double total = 0.0;
+  for (int64_t bg = 0; bg < B * Hkv; ++bg) total += part[bg];
+  free(part);
   if (failed) return ORACLE_ERR_NOMEM;
   if (dscale) *dscale = total;
   return ORACLE_OK;
