@@ -113,6 +113,11 @@ def test_weights_tcgen05_scalar_offset_fill(dtype):
     check(q, k, v, "tcgen05 scalar offset", kernel="weights_tcgen05", is_causal=True, q_offset=40, drop_p=0.1,
           seed=9)
     check(q, k, v, "tcgen05 scalar offset, p = 0", kernel="weights_tcgen05", is_causal=True, q_offset=200)
+    # padding rows (q_lengths) with the statistics pass's fill: zeros, not NaN, past q_len
+    check(q, k, v, "tcgen05 q_lengths, top left", kernel="weights_tcgen05", is_causal=True, q_lengths=[300, 77],
+          drop_p=0.1, seed=10)
+    check(q, k, v, "tcgen05 q_lengths, bottom right", kernel="weights_tcgen05", is_causal="bottom_right",
+          q_lengths=[131, 300], drop_p=0.2, seed=12)
 
 
 def test_weights_causal_gqa_workload_rows():
